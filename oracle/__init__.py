@@ -1,0 +1,278 @@
+"""CPU oracle for the fused FP8 routed-expert MoE forward -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may import this
+package.  The CUDA library (``mixture_experts_fp8_b200``) never imports it and shares no code
+with it.  The arithmetic lives in ``moe_oracle.c`` (plain C, fp64 accumulation, fp32 decisions);
+this module only marshals numpy arrays into it.
+
+Every function cites the page passage it restates in ``moe_oracle.c``:
+  * routing            -- "MindIE-SD Fused MoE", routing selection / parameter table;
+                          "mlx_native ops/moe_gate.rs", moe_gate doc.
+  * permutation        -- "MindIE-SD Fused MoE", execution flow (dispatch, combine).
+  * quantization       -- "metrale_model_layers fp8_grouped_tc_w8a8.rs", module doc (E4M3 per
+                          (row, 128)); "DeepGEMM PR #371", Changes (UE8M0 per 32).
+  * expert MLP, combine -- "metrale ... fp8_grouped_tc_w8a8.rs", run_fp8_grouped_w8a8;
+                          "MATE Mega MoE", API (swiglu) and Current Limits (bf16 output).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "_liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+OK, EINVAL, EUNSUPPORTED = 0, -1, -2
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into _liboracle.so (gcc, OpenMP, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("num_tokens", "hidden", "inter", "num_experts", "top_k", "routing",
+                 "renormalize", "group_count", "k_group", "group_select_mode")] + \
+               [("routed_scaling_factor", ctypes.c_float), ("recipe", ctypes.c_int32)]
+
+
+@dataclass
+class Config:
+    """Problem description; field meanings follow the pages' fused_moe signature."""
+    num_tokens: int
+    hidden: int
+    inter: int
+    num_experts: int
+    top_k: int
+    routing: int = 0             # 0 softmax, 1 sigmoid
+    renormalize: int = 0
+    group_count: int = 1
+    k_group: int = 1
+    group_select_mode: int = 0
+    routed_scaling_factor: float = 1.0
+    recipe: int = 0              # 0 fp32 scale per (row,128); 1 UE8M0 per 32
+
+    @property
+    def group(self) -> int:
+        return 128 if self.recipe == 0 else 32
+
+    @property
+    def scale_dtype(self):
+        return np.float32 if self.recipe == 0 else np.uint8
+
+    def c(self) -> _Cfg:
+        return _Cfg(*(int(getattr(self, n)) for n in
+                      ("num_tokens", "hidden", "inter", "num_experts", "top_k", "routing",
+                       "renormalize", "group_count", "k_group", "group_select_mode")),
+                    float(self.routed_scaling_factor), int(self.recipe))
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            P = ctypes.c_void_p
+            lib.orc_e4m3_decode.restype = ctypes.c_double
+            lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.orc_e4m3_encode.restype = ctypes.c_uint8
+            lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.orc_mx_exponent.restype = ctypes.c_int
+            lib.orc_mx_exponent.argtypes = [ctypes.c_float]
+            lib.orc_bf16_from_double.restype = ctypes.c_uint16
+            lib.orc_bf16_from_double.argtypes = [ctypes.c_double]
+            lib.orc_quant_row.restype = None
+            lib.orc_quant_row.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P]
+            lib.orc_check_cfg.restype = ctypes.c_int
+            lib.orc_check_cfg.argtypes = [ctypes.POINTER(_Cfg)]
+            lib.orc_route.restype = ctypes.c_int
+            lib.orc_route.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P]
+            lib.orc_permute.restype = None
+            lib.orc_permute.argtypes = [ctypes.c_int] * 3 + [P] * 5
+            lib.orc_scaled_gemv.restype = None
+            lib.orc_scaled_gemv.argtypes = [ctypes.c_int] * 3 + [P] * 5
+            lib.orc_forward.restype = ctypes.c_int
+            lib.orc_forward.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 11 + [P, ctypes.c_int, P, P, P]
+            lib.orc_forward_permuted.restype = ctypes.c_int
+            lib.orc_forward_permuted.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 10
+            lib.orc_quantize_tokens.restype = None
+            lib.orc_quantize_tokens.argtypes = [ctypes.c_int] * 3 + [P] * 3
+            lib.orc_num_threads.restype = ctypes.c_int
+            lib.orc_set_num_threads.restype = None
+            lib.orc_set_num_threads.argtypes = [ctypes.c_int]
+            _lib = lib
+    return _lib
+
+
+def _p(a):
+    if a is None:
+        return None
+    assert isinstance(a, np.ndarray) and a.flags["C_CONTIGUOUS"], "need C-contiguous numpy"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _arr(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+# ----------------------------------------------------------------------------- scalar pieces
+def e4m3_decode(code: int) -> float:
+    return _load().orc_e4m3_decode(int(code) & 0xFF)
+
+
+def e4m3_encode(v: float) -> int:
+    return int(_load().orc_e4m3_encode(float(v)))
+
+
+def e4m3_encode_array(x: np.ndarray) -> np.ndarray:
+    lib = _load()
+    flat = np.ascontiguousarray(x, dtype=np.float32).ravel()
+    return np.array([lib.orc_e4m3_encode(float(v)) for v in flat], dtype=np.uint8).reshape(np.shape(x))
+
+
+def mx_exponent(amax: float) -> int:
+    return int(_load().orc_mx_exponent(float(amax)))
+
+
+def bf16_from_double(v: float) -> int:
+    return int(_load().orc_bf16_from_double(float(v)))
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def num_threads() -> int:
+    return int(_load().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    _load().orc_set_num_threads(int(n))
+
+
+# ----------------------------------------------------------------------------- stages
+def quant_row(x: np.ndarray, recipe: int):
+    """Quantize one fp32 row; returns (codes uint8 [n], scales fp32 [n/128] | uint8 [n/32])."""
+    x = _arr(x, np.float32).ravel()
+    n = x.size
+    g = 128 if recipe == 0 else 32
+    q = np.zeros(n, np.uint8)
+    s = np.zeros(n // g, np.float32 if recipe == 0 else np.uint8)
+    _load().orc_quant_row(_p(x), n, recipe, _p(q), _p(s))
+    return q, s
+
+
+def quantize_tokens(x_bf16: np.ndarray, recipe: int):
+    """x bf16 bits uint16 [T,H] -> (codes [T,H], scales [T,H/g])."""
+    x = _arr(x_bf16, np.uint16)
+    T, H = x.shape
+    g = 128 if recipe == 0 else 32
+    q = np.zeros((T, H), np.uint8)
+    s = np.zeros((T, H // g), np.float32 if recipe == 0 else np.uint8)
+    _load().orc_quantize_tokens(T, H, recipe, _p(x), _p(q), _p(s))
+    return q, s
+
+
+def check_cfg(cfg: Config) -> int:
+    c = cfg.c()
+    return int(_load().orc_check_cfg(ctypes.byref(c)))
+
+
+def route(cfg: Config, logits: np.ndarray, per_expert_scale=None):
+    """-> (topk_idx int32 [T,k], topk_weights fp32 [T,k], near_tie uint8 [T])."""
+    logits = _arr(logits, np.float32)
+    pes = _arr(per_expert_scale, np.float32)
+    T, k = cfg.num_tokens, cfg.top_k
+    idx = np.zeros((T, k), np.int32)
+    w = np.zeros((T, k), np.float32)
+    tie = np.zeros(T, np.uint8)
+    c = cfg.c()
+    rc = _load().orc_route(ctypes.byref(c), _p(logits), _p(pes), _p(idx), _p(w), _p(tie))
+    if rc:
+        raise ValueError(f"oracle route: invalid configuration ({rc})")
+    return idx, w, tie
+
+
+def permute(topk_idx: np.ndarray, num_experts: int):
+    """-> (counts [E], offsets [E+1], row_src [A], row_of [T,k]), all int32."""
+    idx = _arr(topk_idx, np.int32)
+    T, k = idx.shape
+    E = num_experts
+    counts = np.zeros(E, np.int32)
+    offsets = np.zeros(E + 1, np.int32)
+    row_src = np.zeros(T * k, np.int32)
+    row_of = np.zeros((T, k), np.int32)
+    _load().orc_permute(T, k, E, _p(idx), _p(counts), _p(offsets), _p(row_src), _p(row_of))
+    return counts, offsets, row_src, row_of
+
+
+def scaled_gemv(recipe: int, aq, as_, wq, ws):
+    """One block-scaled FP8 GEMM row: aq [K] codes, as_ [K/g], wq [K,N] codes, ws [K/g,N]."""
+    aq = _arr(aq, np.uint8).ravel()
+    wq = _arr(wq, np.uint8)
+    sd = np.float32 if recipe == 0 else np.uint8
+    as_ = _arr(as_, sd).ravel()
+    ws = _arr(ws, sd)
+    K, N = wq.shape
+    out = np.zeros(N, np.float64)
+    _load().orc_scaled_gemv(recipe, K, N, _p(aq), _p(as_), _p(wq), _p(ws), _p(out))
+    return out
+
+
+def forward(cfg: Config, x_bf16, w13, w13s, w2, w2s, logits=None, per_expert_scale=None,
+            topk_idx=None, topk_weights=None, b13=None, b2=None, tokens=None,
+            want_act: bool = False):
+    """Full layer forward.  x_bf16 uint16 [T,H]; weights in the pages' layout:
+    w13 uint8 [E,H,2I], w13s [E,H/g,2I]; w2 uint8 [E,I,H], w2s [E,I/g,H]; biases bf16 bits.
+    Returns y bf16 bits uint16 [n_sel,H] (and, with want_act, the per-slot act codes/scales)."""
+    x = _arr(x_bf16, np.uint16)
+    sd = cfg.scale_dtype
+    args = [x, _arr(logits, np.float32), _arr(per_expert_scale, np.float32),
+            _arr(topk_idx, np.int32), _arr(topk_weights, np.float32),
+            _arr(w13, np.uint8), _arr(w13s, sd), _arr(w2, np.uint8), _arr(w2s, sd),
+            _arr(b13, np.uint16), _arr(b2, np.uint16)]
+    tok = _arr(tokens, np.int32)
+    n_sel = cfg.num_tokens if tok is None else int(tok.size)
+    y = np.zeros((n_sel, cfg.hidden), np.uint16)
+    act_q = act_s = None
+    if want_act:
+        act_q = np.zeros((n_sel, cfg.top_k, cfg.inter), np.uint8)
+        act_s = np.zeros((n_sel, cfg.top_k, cfg.inter // cfg.group), sd)
+    c = cfg.c()
+    rc = _load().orc_forward(ctypes.byref(c), *[_p(a) for a in args], _p(tok), n_sel, _p(y),
+                             _p(act_q), _p(act_s))
+    if rc:
+        raise ValueError(f"oracle forward: invalid configuration ({rc})")
+    return (y, act_q, act_s) if want_act else y
+
+
+def forward_permuted(cfg: Config, x_bf16, w13, w13s, w2, w2s, logits, per_expert_scale=None,
+                     b13=None, b2=None):
+    """The same forward computed expert by expert over permuted rows (route, permute, mlp,
+    combine); must agree bit for bit with forward()."""
+    sd = cfg.scale_dtype
+    args = [_arr(x_bf16, np.uint16), _arr(logits, np.float32), _arr(per_expert_scale, np.float32),
+            _arr(w13, np.uint8), _arr(w13s, sd), _arr(w2, np.uint8), _arr(w2s, sd),
+            _arr(b13, np.uint16), _arr(b2, np.uint16)]
+    y = np.zeros((cfg.num_tokens, cfg.hidden), np.uint16)
+    c = cfg.c()
+    rc = _load().orc_forward_permuted(ctypes.byref(c), *[_p(a) for a in args], _p(y))
+    if rc:
+        raise ValueError(f"oracle forward_permuted: invalid configuration ({rc})")
+    return y
