@@ -1,0 +1,381 @@
+"""Benchmark of the fused FP8 routed-expert MoE layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|tiny|prefill|skewed|large]
+                    [--impl reference] [--no-cpu-baseline]
+
+One step = one moe_forward call (route, permute, quantize, gate+up GEMM with SwiGLU and
+requantization, down GEMM, combine) over one batch of seeded synthetic inputs of the named
+problem, inputs resident in HBM.  The default problem is the decode configuration (64 tokens,
+H 2816, I 768, 128 experts, top-8); its ~0.85 GB of FP8 weights exceed the 126 MB L2, so every
+step streams them from HBM.
+
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) are independent replicas, one per
+GPU, with no collective on the data path ("scaling": "weak"); timing is the max over ranks.
+`--impl reference` times the CPU oracle (test infrastructure, plain C) on host cores on a
+bounded token sample of the same problem.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s & FP8 TFLOPS (% of tensor/HBM roofline), 1×B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
+KERNELS_PER_STEP = 8         # route, hist, scan, scatter, quant, gemm1, gemm2, combine
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def describe(shape: synth.Shape) -> str:
+    rt = "sigmoid" if shape.routing else "softmax"
+    extra = []
+    if shape.group_count > 1:
+        extra.append(f"groups {shape.group_count}/{shape.k_group} mode {shape.group_select_mode}")
+    if shape.renormalize:
+        extra.append("renorm")
+    if shape.per_expert_scale:
+        extra.append("per-expert scale")
+    if shape.routed_scaling_factor != 1.0:
+        extra.append(f"rsf {shape.routed_scaling_factor}")
+    if shape.biases:
+        extra.append("biases")
+    rec = "E4M3 + fp32 scale per (row,128)" if shape.recipe == 0 else "MXFP8 (E4M3 + UE8M0 per 32)"
+    return (f"{shape.name}: {shape.num_tokens} tok, H {shape.hidden}, I {shape.inter}, "
+            f"E {shape.num_experts}, top-{shape.top_k}, {rt}" + (", " + ", ".join(extra) if extra else "")
+            + f"; {rec}")
+
+
+def flops(shape, A):
+    return 6.0 * A * shape.hidden * shape.inter
+
+
+def scale_bytes(shape, K, N):
+    return (K // 128) * N * 4 if shape.recipe == 0 else (K // 32) * N
+
+
+def algorithmic_bytes(shape, active):
+    """Minimum HBM bytes of one forward: each active expert's weights and scales once, plus the
+    per-call tensors (x, y, logits).  Intermediates excluded."""
+    H, I, E, T = shape.hidden, shape.inter, shape.num_experts, shape.num_tokens
+    w = active * (3 * H * I + scale_bytes(shape, H, 2 * I) + scale_bytes(shape, I, H))
+    if shape.biases:
+        w += active * 2 * (2 * I + H)
+    return w + 2 * T * H * 2 + 4 * T * E
+
+
+def gemm1_bytes(shape, active):
+    """Algorithmic bytes of one gate+up launch: active experts' W13 codes + scales, the
+    quantized activations read, the requantized SwiGLU products written."""
+    H, I, T, k = shape.hidden, shape.inter, shape.num_tokens, shape.top_k
+    A = T * k
+    g = 128 if shape.recipe == 0 else 32
+    sb = 4 if shape.recipe == 0 else 1
+    return (active * (2 * I * H + scale_bytes(shape, H, 2 * I)) + A * H + A * (H // g) * sb
+            + A * I + A * (I // g) * sb)
+
+
+def gemm2_bytes(shape, active):
+    H, I, T, k = shape.hidden, shape.inter, shape.num_tokens, shape.top_k
+    A = T * k
+    g = 128 if shape.recipe == 0 else 32
+    sb = 4 if shape.recipe == 0 else 1
+    return active * (I * H + scale_bytes(shape, I, H)) + A * I + A * (I // g) * sb + A * H * 4
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms in the background."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index=0):
+        self.proc = None
+        self.t0 = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            uuid = str(getattr(props, "uuid", "")) or None
+            sel = ["-i", ("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else uuid] if uuid else []
+            self.path = os.path.join("/tmp", f"moefp8_clocks_{os.getpid()}.csv")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, f"--query-gpu=timestamp,{self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, window):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait(timeout=5)
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[3:]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        t0, t1 = window
+        sel = [r for r in rows if t0 - 1.0 <= r[0] <= t1 + 1.0] or rows
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in sel for n, v in zip(names, r[3][2:6]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in sel), "sm_max_mhz": max(r[2] for r in sel),
+                "reasons": reasons, "samples": len(sel)}
+
+
+def traffic_for(kernel: str, workload: str):
+    """dram bytes per launch from a committed ncu summary, if it was taken on the current
+    kernel source (matching hash); else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        ent = d.get(f"{kernel}:{workload}")
+        src = os.path.join(ROOT, "mixture_experts_fp8_b200", "csrc", ent["source"])
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        return ent["dram_bytes_per_launch"] if h == ent["source_sha256_16"] else None
+    except Exception:
+        return None
+
+
+def run_cpu_oracle(shape, prob, n_tokens, threads=None):
+    import oracle
+    if threads:
+        oracle.set_num_threads(threads)
+    ni = prob.numpy_inputs()
+    c = oracle.Config(**shape.cfg())
+    tok = np.linspace(0, shape.num_tokens - 1, n_tokens).astype(np.int32)
+    t = time.perf_counter()
+    oracle.forward(c, ni["x"], ni["w13"], ni["w13s"], ni["w2"], ni["w2s"], logits=ni["logits"],
+                   per_expert_scale=ni["per_expert_scale"], b13=ni["b13"], b2=ni["b2"], tokens=tok)
+    dt = time.perf_counter() - t
+    return n_tokens / dt, dt, oracle.num_threads()
+
+
+def reference_arm(args, shape, rank):
+    if rank != 0:
+        return
+    prob = synth.make_problem(shape, device="cpu")
+    n = {"tiny": 16, "decode": 8, "skewed": 16, "prefill": 2, "large": 4}.get(shape.name, 4)
+    for _ in range(args.warmup):
+        run_cpu_oracle(shape, prob, 1)
+    times = []
+    for _ in range(args.steps):
+        _, dt, cores = run_cpu_oracle(shape, prob, n)
+        times.append(dt)
+    tot = sum(times)
+    value = n * args.steps / tot
+    sample = f"{n} of {shape.num_tokens} tokens per step (a row's output does not depend on other rows)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": describe(shape), "tokens_per_step": n},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="decode", choices=sorted(synth.SHAPES))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    shape = synth.SHAPES[args.config]
+
+    if args.impl == "reference":
+        reference_arm(args, shape, rank)
+        return
+
+    import mixture_experts_fp8_b200 as moe
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    dev = f"cuda:{local}"
+    gen_dev = dev if shape.name in ("prefill", "large") else "cpu"
+    prob = synth.make_problem(shape, device=gen_dev)
+    d = prob.to(dev)
+    cfg = moe.Config(**shape.cfg())
+    weights = moe.transform_weights(cfg, d.w13, d.w13_scale, d.w2, d.w2_scale)
+    if shape.name in ("prefill", "large"):
+        del d.w13, d.w2
+    ws = moe.new_workspace(cfg, dev)
+    y = torch.empty((shape.num_tokens, shape.hidden), dtype=torch.bfloat16, device=dev)
+    counts = torch.zeros(shape.num_experts, dtype=torch.int32, device=dev)
+
+    def step(profile=None):
+        moe.forward(cfg, d.x, weights, router_logits=d.logits, per_expert_scale=d.per_expert_scale,
+                    w13_bias=d.w13_bias, w2_bias=d.w2_bias, y=y, expert_counts=counts, workspace=ws,
+                    profile=profile)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = moe.read_status(ws)
+    active = int((counts.cpu() > 0).sum())
+    A = shape.num_tokens * shape.top_k
+
+    prof = moe.Profile()
+    sampler = ClockSampler(local)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record()
+    for _ in range(args.steps):
+        step(prof)
+    end.record()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if dist:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    clocks = sampler.stop((t_wall0, t_wall1))
+    stage_ms, calls = prof.read()
+    prof.close()
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end to end: pinned host inputs -> device, forward, result -> host, every step
+    x_h = d.x.cpu().pin_memory()
+    l_h = d.logits.cpu().pin_memory()
+    y_h = torch.empty_like(y, device="cpu").pin_memory()
+    x_d, l_d = torch.empty_like(d.x), torch.empty_like(d.logits)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        l_d.copy_(l_h, non_blocking=True)
+        moe.forward(cfg, x_d, weights, router_logits=l_d, per_expert_scale=d.per_expert_scale,
+                    w13_bias=d.w13_bias, w2_bias=d.w2_bias, y=y, workspace=ws)
+        y_h.copy_(y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+
+    if rank == 0:
+        pk, pk_kind = peaks()
+        hbm = float(pk["hbm_gbs"])
+        fp8_peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])) * FP8_OVER_BF16
+        tok_s = world * shape.num_tokens * args.steps / (ms / 1e3)
+        per_step_s = ms / 1e3 / args.steps
+        fl = flops(shape, A)
+        alg = algorithmic_bytes(shape, active)
+        g1_ms = stage_ms["gemm1_swiglu_requant"] / max(calls, 1)
+        g2_ms = stage_ms["gemm2"] / max(calls, 1)
+        g1_bytes = gemm1_bytes(shape, active)
+        g1_gbs = g1_bytes / (g1_ms / 1e3) / 1e9
+        g1_tflops = 2.0 * A * shape.hidden * 2 * shape.inter / (g1_ms / 1e3) / 1e12
+        compute_bound = fl / alg > (fp8_peak * 1e12) / (hbm * 1e9)
+        if compute_bound:
+            roof = {"bound": "tensor", "achieved": g1_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                    "frac": g1_tflops / fp8_peak}
+        else:
+            roof = {"bound": "hbm", "achieved": g1_gbs, "peak": hbm, "unit": "GB/s", "frac": g1_gbs / hbm}
+        roof.update({"kernel": "k_grouped_gemm<gate+up>", "traffic": traffic_for("gemm1", shape.name),
+                     "peak_source": f"{pk_kind} ({'sustained bf16 x2 for fp8' if compute_bound else 'copy'})",
+                     "algorithmic_bytes_per_launch": g1_bytes, "ms_per_launch": g1_ms})
+        layer_roof_s = max(fl / (fp8_peak * 1e12), alg / (hbm * 1e9))
+        line = {
+            "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+            "config": {"workload": describe(shape), "tokens_per_step": shape.num_tokens,
+                       "active_experts": active, "parallelism": f"replicas x{world}",
+                       "l2": "no flush; the step streams the FP8 weights, larger than L2" if alg > 126e6
+                             else "working set fits L2 (latency-bound)"},
+            "tflops": fl / per_step_s / 1e12,
+            "layer_roofline": {"bound": "tensor" if compute_bound else "hbm", "roofline_ms": layer_roof_s * 1e3,
+                               "frac": layer_roof_s / per_step_s, "algorithmic_bytes": alg, "flops": fl},
+            "roofline": roof,
+            "stages_ms": {k: v / max(calls, 1) for k, v in stage_ms.items()},
+            "gemm2": {"ms": g2_ms, "GB/s": gemm2_bytes(shape, active) / (g2_ms / 1e3) / 1e9},
+            "clocks": clocks, "gpu_launches": KERNELS_PER_STEP * args.steps, "status": status,
+            "e2e": {"value": world * shape.num_tokens * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": x_h.numel() * 2 + l_h.numel() * 4,
+                    "d2h_bytes_per_step": y_h.numel() * 2},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            n = {"tiny": 16, "decode": 64, "skewed": 64, "prefill": 4, "large": 16}.get(shape.name, 8)
+            cpu_prob = prob if prob.x.device.type == "cpu" else None
+            if cpu_prob is not None:
+                done = tot = 0.0
+                reps = 0
+                while tot < 5.0 and reps < 50:
+                    v, dt, cores = run_cpu_oracle(shape, cpu_prob, n)
+                    tot += dt
+                    done += n
+                    reps += 1
+                line["cpu_baseline"] = {"value": done / tot, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                        "sample": f"{n} of {shape.num_tokens} tokens x {reps} runs, {tot:.1f} s"}
+            else:
+                line["cpu_baseline"] = None
+        print(json.dumps(line), flush=True)
+
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,203 @@
+/*
+ * moefp8.h -- C ABI of libmoefp8.so: the forward of one fused routed-expert FP8 MoE layer on a
+ * single NVIDIA B200 (sm_100a).
+ *
+ * The layer (sources are web pages, cited by title and section):
+ *   "MindIE-SD Fused MoE" -- function signature and parameter table (hidden_states,
+ *       router_logits, num_experts, top_k, w13 [E, hidden, 2*inter], w2 [E, inter, hidden],
+ *       biases, weight scales, k_group / group_count / group_select_mode, routing_method,
+ *       renormalize, routed_scaling_factor, custom_routing_function); execution flow
+ *       (select_experts -> dispatch -> mlp -> combine); routing selection; MXFP8 example.
+ *   "MATE Mega MoE" -- Typical Flow (a caller-owned runtime workspace, a one-time weight
+ *       transform, then the fused expert compute), Current Limits, API (swiglu).
+ *   "metrale_model_layers fp8_grouped_tc_w8a8.rs" -- the W8A8 step: activations quantized to
+ *       E4M3 per (row, 128 group), FP8 weights in E4M3 tensor-core MMAs, SiLU products
+ *       requantized, then the down projection; nothing launches unless the shapes fit.
+ *   "DeepGEMM PR #371: Add W8A8 (FP8xFP8) Mega MoE support" -- UE8M0 scale factors per 32
+ *       elements, 4 packed per 32-bit word; hidden / intermediate sizes that are not multiples
+ *       of 512 (e.g. 768 and 1152).
+ *   "mlx_native ops/moe_gate.rs" -- top-K + softmax + per_expert_scale; output expert ids and
+ *       fp32 weights [T, k]; argument validation with an error message.
+ *
+ * Conventions for every entry point:
+ *   - All tensors are row-major and contiguous; "device" pointers are CUDA device memory of the
+ *     current device, "host" pointers are ordinary host memory.
+ *   - The caller owns every buffer.  The library allocates no device memory and never
+ *     synchronizes the stream, except where an entry point says so.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); all work is enqueued on it
+ *     and runs asynchronously.
+ *   - Return value: MOE_OK, or a negative MOE_ERR_* code.  On an error, nothing is launched and
+ *     moe_last_error() (per host thread) describes the first problem found.
+ *   - Faults found on the device (a bounded wait that ran out, an index out of range) do not
+ *     trap; they are written to the workspace status word, readable with moe_read_status().
+ */
+#ifndef MOEFP8_H
+#define MOEFP8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)   /* a dimension <= 0, top_k outside [1, E], NULL pointer, small buffer */
+#define MOE_ERR_UNSUPPORTED (-2)   /* a valid problem outside what this library implements */
+#define MOE_ERR_CUDA (-3)          /* a CUDA runtime call failed */
+#define MOE_ERR_TIMEOUT (-4)       /* device status: a bounded wait inside a kernel ran out */
+#define MOE_ERR_BOUNDS (-5)        /* device status: an index read from memory was out of range */
+
+#define MOE_MAX_EXPERTS 256
+
+/* One problem.  All fields are validated on every call; the library keeps no global state.
+ *   routing            0 = softmax, 1 = sigmoid  ("MindIE-SD Fused MoE", routing_method)
+ *   renormalize        softmax only: divide the selected weights by their sum; sigmoid
+ *                      weights are always normalized over the selected experts
+ *   group_count        experts form this many contiguous groups (1 = no grouped routing)
+ *   k_group            groups kept per token, in [1, group_count]
+ *   group_select_mode  group score: 0 = max score in the group, 1 = sum of its two largest
+ *   routed_scaling_factor  multiplies every routing weight (applied last)
+ *   recipe             0 = E4M3 with an fp32 scale per (row, 128-element block) for
+ *                          activations and per (output column, 128-deep K block) for weights
+ *                      1 = MXFP8: E4M3 with a UE8M0 power-of-two scale per 32 elements
+ * Limits (MOE_ERR_UNSUPPORTED): hidden % 128, inter % 128, num_experts <= 256,
+ * num_experts % group_count, k_group in [1, group_count], top_k <= k_group * experts per
+ * group, group_select_mode 1 needs >= 2 experts per group.  ("MATE Mega MoE", Current Limits
+ * asks hidden % 128 and inter % 256; inter % 128 is accepted here, as the DeepGEMM PR's
+ * unaligned sizes such as inter = 1152 require.) */
+typedef struct {
+    int32_t num_tokens, hidden, inter, num_experts, top_k;
+    int32_t routing;
+    int32_t renormalize;
+    int32_t group_count, k_group, group_select_mode;
+    float routed_scaling_factor;
+    int32_t recipe;
+} moe_config_t;
+
+/* Byte offsets of the regions inside a forward workspace (for tests and diagnostics).
+ * A = num_tokens * top_k routed rows; g = 128 (recipe 0) or 32 (recipe 1); scales are fp32
+ * (recipe 0) or UE8M0 bytes (recipe 1).  All offsets are multiples of 1024. */
+typedef struct {
+    size_t status;       /* int32 status word (MOE_OK or a device MOE_ERR_*)             */
+    size_t topk_idx;     /* int32 [T, k]   routing computed by moe_forward               */
+    size_t topk_weights; /* fp32  [T, k]                                                 */
+    size_t counts;       /* int32 [E]      routed rows per expert                        */
+    size_t offsets;      /* int32 [E + 1]  first permuted row of each expert             */
+    size_t tile_start;   /* int32 [E + 1]  first 128-row M tile of each expert           */
+    size_t row_src;      /* int32 [A]      permuted row r came from routed row t*k + j   */
+    size_t row_of;       /* int32 [T, k]   permuted row of routed row (t, j)             */
+    size_t hist;         /* int32 [chunks, E] per-chunk expert histograms                */
+    size_t xq;           /* E4M3  [A, H]   quantized activations in permuted order       */
+    size_t xs;           /* scale [A, H/g]                                               */
+    size_t act_q;        /* E4M3  [A, I]   requantized SwiGLU products                   */
+    size_t act_s;        /* scale [A, I/g]                                               */
+    size_t o;            /* fp32  [A, H]   down-projection output per permuted row       */
+    size_t total;        /* bytes the workspace needs                                    */
+} moe_workspace_layout_t;
+
+/* Opaque per-stage timer (CUDA events) for moe_forward_profiled. */
+typedef struct moe_profile moe_profile_t;
+
+#define MOE_NUM_STAGES 6   /* route, permute, quantize, gemm1+swiglu+requant, gemm2, combine */
+
+/* Message for the last error returned on this host thread ("" if none). */
+const char *moe_last_error(void);
+
+/* Validate a configuration without launching anything.  Returns MOE_OK or the error code the
+ * other entry points would return for it. */
+int moe_check_config(const moe_config_t *cfg);
+
+/* Sizes, in bytes, of the four transformed-weight buffers that moe_transform_weights fills
+ * (host call, no CUDA work). */
+int moe_transformed_weights_size(const moe_config_t *cfg, size_t *w13_bytes, size_t *w13s_bytes,
+                                 size_t *w2_bytes, size_t *w2s_bytes);
+
+/* Re-lay the grouped FP8 expert weights for the forward ("MATE Mega MoE", Typical Flow step 2
+ * and transform_weights_for_mega_moe).  Runs once, offline; deterministic and re-runnable.
+ *   w13        device, E4M3 codes [E, H, 2I] (K rows x N columns; columns 0:I gate, I:2I up)
+ *   w13_scale  device, recipe 0: fp32 [E, H/128, 2I]; recipe 1: UE8M0 bytes [E, H/32, 2I]
+ *   w2         device, E4M3 codes [E, I, H]
+ *   w2_scale   device, recipe 0: fp32 [E, I/128, H];  recipe 1: UE8M0 bytes [E, I/32, H]
+ * (scales are K-block-major, the orientation of the "MindIE-SD Fused MoE" MXFP8 example.)
+ * Outputs (device, sizes from moe_transformed_weights_size; opaque to the caller): K-major
+ * codes with gate/up columns interleaved in 64-column blocks, and the scales re-laid to match.
+ * Inputs and outputs must not overlap. */
+int moe_transform_weights(const moe_config_t *cfg, const void *w13, const void *w13_scale,
+                          const void *w2, const void *w2_scale, void *w13_t, void *w13s_t,
+                          void *w2_t, void *w2s_t, void *stream);
+
+/* Workspace bytes moe_forward needs for cfg->num_tokens tokens (host call).  A workspace sized
+ * for T tokens serves every call with num_tokens <= T and the other fields equal.  Like
+ * get_symm_buffer_for_mega_moe ("MATE Mega MoE", API), but on one GPU. */
+int moe_workspace_size(const moe_config_t *cfg, size_t *bytes);
+
+/* Region offsets of that workspace (host call). */
+int moe_workspace_layout(const moe_config_t *cfg, moe_workspace_layout_t *layout);
+
+/* Router top-k alone ("MindIE-SD Fused MoE", select_experts and routing selection;
+ * "mlx_native ops/moe_gate.rs", output ids and weights).
+ *   router_logits     device fp32 [T, E]
+ *   per_expert_scale  device fp32 [E] or NULL (multiplies each selected expert's weight)
+ *   topk_idx          device int32 [T, k]  out: expert ids, best first; ties -> lower index
+ *   topk_weights      device fp32  [T, k]  out: routing weights                          */
+int moe_route(const moe_config_t *cfg, const float *router_logits, const float *per_expert_scale,
+              int32_t *topk_idx, float *topk_weights, void *stream);
+
+/* The fused layer forward ("MindIE-SD Fused MoE", fused_moe; "MATE Mega MoE",
+ * fp8_fp8_mega_moe): route -> permute -> quantize -> gate+up GEMM with SwiGLU and
+ * requantization -> down GEMM -> weighted combine.
+ *   hidden_states     device bf16 [T, H]
+ *   router_logits     device fp32 [T, E], or NULL when topk_idx/topk_weights are given
+ *   per_expert_scale  device fp32 [E] or NULL (used only with router_logits)
+ *   topk_idx          device int32 [T, k] or NULL: routing supplied by the caller (the
+ *   topk_weights      device fp32  [T, k]  custom routing function path); exactly one of
+ *                                           router_logits and topk_idx must be non-NULL.
+ *                                           The k ids of a token must be distinct, in [0, E).
+ *   w13_t .. w2s_t    device, from moe_transform_weights with the same cfg fields
+ *   w13_bias          device bf16 [E, 2I] or NULL
+ *   w2_bias           device bf16 [E, H] or NULL
+ *   y                 device bf16 [T, H], contiguous; out
+ *   expert_counts     device int32 [E] or NULL; out: rows routed to each expert
+ *   workspace         device, >= moe_workspace_size bytes, 1024-byte aligned; scratch owned by
+ *                     the caller; must not be shared by calls in flight at the same time
+ * A row's output bits do not depend on the other rows of the batch. */
+int moe_forward(const moe_config_t *cfg, const void *hidden_states, const float *router_logits,
+                const float *per_expert_scale, const int32_t *topk_idx, const float *topk_weights,
+                const void *w13_t, const void *w13s_t, const void *w2_t, const void *w2s_t,
+                const void *w13_bias, const void *w2_bias, void *y, int32_t *expert_counts,
+                void *workspace, size_t workspace_bytes, void *stream);
+
+/* moe_forward, recording a CUDA event before each of the MOE_NUM_STAGES stages and after the
+ * last one into `prof` (which accumulates per-stage device time until reset).  prof may be
+ * NULL, which makes this identical to moe_forward. */
+int moe_forward_profiled(const moe_config_t *cfg, const void *hidden_states,
+                         const float *router_logits, const float *per_expert_scale,
+                         const int32_t *topk_idx, const float *topk_weights, const void *w13_t,
+                         const void *w13s_t, const void *w2_t, const void *w2s_t,
+                         const void *w13_bias, const void *w2_bias, void *y,
+                         int32_t *expert_counts, void *workspace, size_t workspace_bytes,
+                         moe_profile_t *prof, void *stream);
+
+/* Create / destroy a stage profiler (creates CUDA events on the current device). */
+int moe_profile_create(moe_profile_t **prof);
+int moe_profile_destroy(moe_profile_t *prof);
+/* Synchronize on the recorded events, add their elapsed times into the totals and return the
+ * totals: stage_ms[MOE_NUM_STAGES] (milliseconds summed over calls) and *calls. */
+int moe_profile_read(moe_profile_t *prof, float *stage_ms, int32_t *calls);
+int moe_profile_reset(moe_profile_t *prof);
+
+/* Read the workspace status word (blocking copy after synchronizing `stream`): MOE_OK, or
+ * MOE_ERR_TIMEOUT / MOE_ERR_BOUNDS set by a kernel.  moe_forward clears it when it starts. */
+int moe_read_status(const void *workspace, int32_t *status, void *stream);
+
+/* Failure-detection self test: launch one kernel that waits on a barrier nothing will ever
+ * complete, with a limit of `timeout_us` microseconds, after which it writes MOE_ERR_TIMEOUT to
+ * the device int32 *status and returns.  The context stays usable. */
+int moe_selftest_bounded_wait(int32_t *status, uint32_t timeout_us, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEFP8_H */

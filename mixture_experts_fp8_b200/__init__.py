@@ -1,0 +1,272 @@
+"""mixture_experts_fp8_b200 -- a B200-native fused FP8 routed-expert MoE layer (forward).
+
+Thin Python binding over ``libmoefp8.so`` (C ABI in ``include/moefp8.h``).  This module only
+marshals arguments: every step of the layer runs in the library's sm_100a kernels.  PyTorch
+supplies device memory and streams.  There is no CPU fallback: if the library is missing it is
+built in-tree with nvcc, and if that is impossible, importing this package fails.
+
+Entry points (same names as the C ABI):
+    check_config, transformed_weights_size, transform_weights, workspace_size,
+    workspace_layout, route, forward, forward_profiled, read_status, selftest_bounded_wait,
+    Profile (moe_profile_create / read / reset / destroy).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import asdict, dataclass
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoefp8.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED = -2
+MOE_ERR_CUDA = -3
+MOE_ERR_TIMEOUT = -4
+MOE_ERR_BOUNDS = -5
+MOE_NUM_STAGES = 6
+STAGE_NAMES = ("route", "permute", "quantize", "gemm1_swiglu_requant", "gemm2", "combine")
+
+EXPORTED = (
+    "moe_last_error", "moe_check_config", "moe_transformed_weights_size", "moe_transform_weights",
+    "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_forward", "moe_forward_profiled",
+    "moe_profile_create", "moe_profile_destroy", "moe_profile_read", "moe_profile_reset",
+    "moe_read_status", "moe_selftest_bounded_wait",
+)
+
+
+class MoeError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("num_tokens", "hidden", "inter", "num_experts", "top_k", "routing",
+                 "renormalize", "group_count", "k_group", "group_select_mode")] + \
+               [("routed_scaling_factor", ctypes.c_float), ("recipe", ctypes.c_int32)]
+
+
+_LAYOUT_FIELDS = ("status", "topk_idx", "topk_weights", "counts", "offsets", "tile_start",
+                  "row_src", "row_of", "hist", "xq", "xs", "act_q", "act_s", "o", "total")
+
+
+class _Layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in _LAYOUT_FIELDS]
+
+
+@dataclass
+class Config:
+    """One problem (moe_config_t).  routing: 0 softmax, 1 sigmoid; recipe: 0 fp32 scale per
+    (row, 128), 1 MXFP8 (UE8M0 per 32)."""
+    num_tokens: int
+    hidden: int
+    inter: int
+    num_experts: int
+    top_k: int
+    routing: int = 0
+    renormalize: int = 0
+    group_count: int = 1
+    k_group: int = 1
+    group_select_mode: int = 0
+    routed_scaling_factor: float = 1.0
+    recipe: int = 0
+
+    def c(self) -> _Cfg:
+        d = asdict(self)
+        return _Cfg(*(int(d[n]) for n in ("num_tokens", "hidden", "inter", "num_experts", "top_k",
+                                          "routing", "renormalize", "group_count", "k_group",
+                                          "group_select_mode")),
+                    float(d["routed_scaling_factor"]), int(d["recipe"]))
+
+    @property
+    def group(self) -> int:
+        return 128 if self.recipe == 0 else 32
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            from . import build as _build
+            _build.build()
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libmoefp8.so is missing and could not be built")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        CP = ctypes.POINTER(_Cfg)
+        lib.moe_last_error.restype = ctypes.c_char_p
+        lib.moe_last_error.argtypes = []
+        sig = {
+            "moe_check_config": [CP],
+            "moe_transformed_weights_size": [CP, ctypes.POINTER(S), ctypes.POINTER(S),
+                                             ctypes.POINTER(S), ctypes.POINTER(S)],
+            "moe_transform_weights": [CP] + [P] * 9,
+            "moe_workspace_size": [CP, ctypes.POINTER(S)],
+            "moe_workspace_layout": [CP, ctypes.POINTER(_Layout)],
+            "moe_route": [CP, P, P, P, P, P],
+            "moe_forward": [CP] + [P] * 14 + [S, P],
+            "moe_forward_profiled": [CP] + [P] * 14 + [S, P, P],
+            "moe_profile_create": [ctypes.POINTER(P)],
+            "moe_profile_destroy": [P],
+            "moe_profile_read": [P, P, P],
+            "moe_profile_reset": [P],
+            "moe_read_status": [P, P, P],
+            "moe_selftest_bounded_wait": [P, ctypes.c_uint32, P],
+        }
+        for name, args in sig.items():
+            f = getattr(lib, name)
+            f.restype = I
+            f.argtypes = args
+        _lib = lib
+        return lib
+
+
+def lib():
+    return _load()
+
+
+def _check(rc: int):
+    if rc != MOE_OK:
+        raise MoeError(rc, _load().moe_last_error().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# --------------------------------------------------------------------------------------------
+def check_config(cfg: Config) -> None:
+    c = cfg.c()
+    _check(_load().moe_check_config(ctypes.byref(c)))
+
+
+def transformed_weights_size(cfg: Config):
+    c = cfg.c()
+    out = [ctypes.c_size_t() for _ in range(4)]
+    _check(_load().moe_transformed_weights_size(ctypes.byref(c), *[ctypes.byref(o) for o in out]))
+    return tuple(o.value for o in out)
+
+
+def transform_weights(cfg: Config, w13, w13_scale, w2, w2_scale, stream=None):
+    """Device tensors in the pages' layout -> (w13_t, w13s_t, w2_t, w2s_t) uint8 device tensors."""
+    import torch
+    sizes = transformed_weights_size(cfg)
+    outs = [torch.empty(n, dtype=torch.uint8, device=w13.device) for n in sizes]
+    c = cfg.c()
+    _check(_load().moe_transform_weights(ctypes.byref(c), _ptr(w13), _ptr(w13_scale), _ptr(w2),
+                                         _ptr(w2_scale), *[_ptr(o) for o in outs], _stream(stream)))
+    return tuple(outs)
+
+
+def workspace_size(cfg: Config) -> int:
+    c = cfg.c()
+    n = ctypes.c_size_t()
+    _check(_load().moe_workspace_size(ctypes.byref(c), ctypes.byref(n)))
+    return n.value
+
+
+def workspace_layout(cfg: Config) -> dict:
+    c = cfg.c()
+    L = _Layout()
+    _check(_load().moe_workspace_layout(ctypes.byref(c), ctypes.byref(L)))
+    return {n: getattr(L, n) for n in _LAYOUT_FIELDS}
+
+
+def new_workspace(cfg: Config, device="cuda"):
+    import torch
+    return torch.empty(workspace_size(cfg), dtype=torch.uint8, device=device)
+
+
+def route(cfg: Config, router_logits, per_expert_scale=None, topk_idx=None, topk_weights=None,
+          stream=None):
+    """-> (topk_idx int32 [T,k], topk_weights fp32 [T,k]) on the logits' device."""
+    import torch
+    T, k = cfg.num_tokens, cfg.top_k
+    if topk_idx is None:
+        topk_idx = torch.empty((T, k), dtype=torch.int32, device=router_logits.device)
+    if topk_weights is None:
+        topk_weights = torch.empty((T, k), dtype=torch.float32, device=router_logits.device)
+    c = cfg.c()
+    _check(_load().moe_route(ctypes.byref(c), _ptr(router_logits), _ptr(per_expert_scale),
+                             _ptr(topk_idx), _ptr(topk_weights), _stream(stream)))
+    return topk_idx, topk_weights
+
+
+def forward(cfg: Config, hidden_states, weights, router_logits=None, per_expert_scale=None,
+            topk_idx=None, topk_weights=None, w13_bias=None, w2_bias=None, y=None,
+            expert_counts=None, workspace=None, stream=None, profile: "Profile | None" = None):
+    """The fused layer forward.  `weights` = (w13_t, w13s_t, w2_t, w2s_t) from
+    transform_weights.  Returns y (bf16 [T, H])."""
+    import torch
+    if y is None:
+        y = torch.empty((cfg.num_tokens, cfg.hidden), dtype=torch.bfloat16, device=hidden_states.device)
+    if workspace is None:
+        workspace = new_workspace(cfg, hidden_states.device)
+    c = cfg.c()
+    args = [ctypes.byref(c), _ptr(hidden_states), _ptr(router_logits), _ptr(per_expert_scale),
+            _ptr(topk_idx), _ptr(topk_weights), *[_ptr(w) for w in weights], _ptr(w13_bias),
+            _ptr(w2_bias), _ptr(y), _ptr(expert_counts), _ptr(workspace),
+            ctypes.c_size_t(workspace.numel() * workspace.element_size())]
+    if profile is None:
+        _check(_load().moe_forward(*args, _stream(stream)))
+    else:
+        _check(_load().moe_forward_profiled(*args, profile.handle, _stream(stream)))
+    return y
+
+
+def read_status(workspace, stream=None) -> int:
+    st = ctypes.c_int32()
+    _check(_load().moe_read_status(_ptr(workspace), ctypes.byref(st), _stream(stream)))
+    return st.value
+
+
+def selftest_bounded_wait(status_tensor, timeout_us: int, stream=None) -> None:
+    _check(_load().moe_selftest_bounded_wait(_ptr(status_tensor), int(timeout_us), _stream(stream)))
+
+
+class Profile:
+    """Per-stage device time of moe_forward_profiled calls (CUDA events inside the library)."""
+
+    def __init__(self):
+        h = ctypes.c_void_p()
+        _check(_load().moe_profile_create(ctypes.byref(h)))
+        self.handle = h
+
+    def read(self):
+        ms = (ctypes.c_float * MOE_NUM_STAGES)()
+        calls = ctypes.c_int32()
+        _check(_load().moe_profile_read(self.handle, ms, ctypes.byref(calls)))
+        return dict(zip(STAGE_NAMES, list(ms))), calls.value
+
+    def reset(self):
+        _check(_load().moe_profile_reset(self.handle))
+
+    def close(self):
+        if self.handle:
+            _load().moe_profile_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

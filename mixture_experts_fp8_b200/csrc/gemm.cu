@@ -1,0 +1,416 @@
+// gemm.cu -- grouped, block-scaled FP8 GEMM on the 5th-generation tensor cores (tcgen05), for
+// both expert projections of the layer.
+//
+//   mode 0 (gate+up): h[r, n] = sum_g a_s[r,g] * w_s[e,g,n] * sum_{k in g} xq[r,k] * w13[e,n,k]
+//                     (+ b13), then act = silu(h_gate) * h_up, requantized per (row, g)
+//   mode 1 (down):    o[r, n] = sum_g ... act_q[r,k] * w2[e,n,k] (+ b2), stored fp32
+// for every permuted row r of expert e.  "metrale_model_layers fp8_grouped_tc_w8a8.rs",
+// run_fp8_grouped_w8a8: the FP8 weights go into E4M3 tensor-core MMAs undecoded, gate+up writes
+// quantized SiLU products, then the down projection; "MATE Mega MoE", API: swiglu;
+// "MindIE-SD Fused MoE", parameter table: w13_bias / w2_bias.
+//
+// Design (one persistent CTA per SM, 320 threads):
+//   warp 0   TMA producer: per 128-deep K stage, a 128x128 A tile and a 256x128 B tile (both
+//            K-major, 128-byte swizzle) plus the 256 weight scales of the stage (bulk copy).
+//   warp 1   MMA issuer (one thread): tcgen05.mma.kind::f8f6f4, M=128 N=256 K=32.  Each scale
+//            group (128 deep for recipe 0, 32 for recipe 1) is accumulated alone into one of two
+//            256-column fp32 TMEM buffers.
+//   warps 2-9 epilogue: a warp reads its 32 TMEM lanes (= tile rows), half of the columns each;
+//            every group partial is multiplied by a_s * w_s and added into fp32 registers (the
+//            "promotion"), then the tile's epilogue runs from registers.
+// Work unit = (expert, 256-column block, 128-row block), enumerated expert by expert, column
+// block, then row block; CTA c takes units c, c + grid, ...  Rows past an expert's end are
+// computed on whatever the tile holds and never stored.  Every wait is bounded.
+#include <math.h>
+
+#include "moe_common.cuh"
+#include "moe_kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kABytes = kTileM * kTileK;      // 16 KB
+constexpr uint32_t kBBytes = kTileN * kTileK;      // 32 KB
+constexpr uint32_t kWsBytes = kTileN * 4;          // fp32 or 4 x UE8M0 per column
+constexpr uint32_t kTmemCols = 2 * kTileN;         // two fp32 accumulators
+constexpr unsigned long long kDrainLimitNs = 100000000ull;
+
+struct L {
+    static constexpr uint32_t a = 0;
+    static constexpr uint32_t b = a + kStages * kABytes;
+    static constexpr uint32_t ws = b + kStages * kBBytes;
+    static constexpr uint32_t bars = ws + kStages * kWsBytes;
+    static constexpr uint32_t nbars = 2 * kStages + 7;   // full, empty, tfull[2], tempty[2], drain, amax[2]
+    static constexpr uint32_t misc = bars + nbars * 8;   // tmem holder, abort flag
+    static constexpr uint32_t amax = misc + 16;          // float [2 buffers][2 halves][128 rows]
+    static constexpr uint32_t tstart = amax + 2 * 2 * 128 * 4;
+    static constexpr uint32_t off = tstart + (MOE_MAX_EXPERTS + 1) * 4;
+    static constexpr uint32_t end = off + (MOE_MAX_EXPERTS + 1) * 4;
+};
+constexpr uint32_t kSmemBytes = L::end + 1024;   // + slack to align the base to 1024 bytes
+
+// Bounded wait used only while leaving after an abort: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, parity))
+        if (globaltimer_ns() - t0 > kDrainLimitNs) break;
+}
+
+// Unit u -> (expert e, column block nb, row block mb).  Expert e owns units
+// [nt * tstart[e], nt * tstart[e+1]); empty experts own none.
+__device__ __forceinline__ void decode_unit(int u, int nt, const int* tstart, int E, int& e, int& nb,
+                                            int& mb) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (nt * tstart[mid] <= u) lo = mid;
+        else hi = mid - 1;
+    }
+    e = lo;
+    const int local = u - nt * tstart[e];
+    const int mt = tstart[e + 1] - tstart[e];
+    nb = local / mt;
+    mb = local - nb * mt;
+}
+
+// acc[j] += P[j] * (sa * ws[j]) for the 128 columns of this thread's half.
+__device__ __forceinline__ void promote_fp32(float (&acc)[128], uint32_t taddr, const float* ws, float sa) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint32_t v[16];
+        MOE_TMEM_LD16(taddr + c * 16, v);
+        MOE_TMEM_WAIT_LD16(v);
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(ws + c * 16 + j);
+            acc[c * 16 + j + 0] = fmaf(__uint_as_float(v[j + 0]), sa * w4.x, acc[c * 16 + j + 0]);
+            acc[c * 16 + j + 1] = fmaf(__uint_as_float(v[j + 1]), sa * w4.y, acc[c * 16 + j + 1]);
+            acc[c * 16 + j + 2] = fmaf(__uint_as_float(v[j + 2]), sa * w4.z, acc[c * 16 + j + 2]);
+            acc[c * 16 + j + 3] = fmaf(__uint_as_float(v[j + 3]), sa * w4.w, acc[c * 16 + j + 3]);
+        }
+    }
+}
+
+// Same with UE8M0 scales: the scale is 2^(ea + ew - 254), exact.
+__device__ __forceinline__ void promote_mx(float (&acc)[128], uint32_t taddr, const uint32_t* ws4, int ea,
+                                           int g) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint32_t v[16];
+        MOE_TMEM_LD16(taddr + c * 16, v);
+        MOE_TMEM_WAIT_LD16(v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int ew = static_cast<int>((ws4[c * 16 + j] >> (8 * g)) & 0xFFu);
+            acc[c * 16 + j] = fmaf(__uint_as_float(v[j]), exp2_int(ea + ew - 254), acc[c * 16 + j]);
+        }
+    }
+}
+
+}  // namespace
+
+template <int MODE, int RECIPE>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    const int nt = (p.N + kTileN - 1) / kTileN;
+    const int total_units = p.tile_start[p.E] * nt;
+    if (static_cast<int>(blockIdx.x) >= total_units) return;
+
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::bars);
+    uint64_t* empty = full + kStages;
+    uint64_t* tfull = empty + kStages;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint64_t* amax_bar = drain + 1;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::misc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc + 4);
+    float* s_amax = reinterpret_cast<float*>(smem + L::amax);
+    int* s_tstart = reinterpret_cast<int*>(smem + L::tstart);
+    int* s_off = reinterpret_cast<int*>(smem + L::off);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i <= p.E; i += kThreads) {
+        s_tstart[i] = p.tile_start[i];
+        s_off[i] = p.offsets[i];
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1 + kEpiWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], kEpiWarps);
+            mbar_init(&amax_bar[b], kEpiWarps);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    const int KB = p.K / kTileK;                 // pipeline stages per unit
+    constexpr int GPS = RECIPE == 0 ? 1 : 4;     // scale groups per stage
+    constexpr int MPG = 4 / GPS;                 // K=32 MMAs per scale group
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+                int e, nb, mb;
+                decode_unit(u, nt, s_tstart, p.E, e, nb, mb);
+                const int row0 = s_off[e] + mb * kTileM;
+                const int brow0 = e * p.N + nb * kTileN;
+                const uint32_t ws_bytes = static_cast<uint32_t>(min(kTileN, p.N - nb * kTileN)) * 4u;
+                const uint8_t* ws_src = static_cast<const uint8_t*>(p.w_scale) +
+                                        (static_cast<size_t>(e) * KB * p.N + static_cast<size_t>(nb) * kTileN) * 4;
+                for (int kb = 0; kb < KB; ++kb, ++it) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + ws_bytes);
+                    tma_load_2d(smem + L::a + s * kABytes, &tmA, kb * kTileK, row0, &full[s]);
+                    tma_load_2d(smem + L::b + s * kBBytes, &tmB, kb * kTileK, brow0, &full[s]);
+                    bulk_load(smem + L::ws + s * kWsBytes, ws_src + static_cast<size_t>(kb) * p.N * 4, ws_bytes,
+                              &full[s]);
+                }
+            }
+            if (!ok) {   // let the copies already issued land before the CTA leaves
+                const uint32_t n = it < static_cast<uint32_t>(kStages) ? it : kStages;
+                for (uint32_t i = it - n; i < it; ++i) drain_wait(&full[i % kStages], (i / kStages) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = f8_idesc(kTileM, kTileN);
+            uint32_t it = 0, kg = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+                for (int kb = 0; kb < KB && ok; ++kb, ++it) {
+                    const int s = it % kStages;
+                    if (!mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + L::a + s * kABytes);
+                    const uint32_t b_addr = smem_u32(smem + L::b + s * kBBytes);
+                    for (int g = 0; g < GPS; ++g, ++kg) {
+                        const int b = kg & 1;
+                        if (!mbar_wait(&tempty[b], ((kg >> 1) & 1) ^ 1, abort_flag, p.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d = tmem_base + static_cast<uint32_t>(b * kTileN);
+                        for (int m = 0; m < MPG; ++m) {
+                            const uint32_t koff = static_cast<uint32_t>((g * MPG + m) * 32);
+                            mma_f8(d, sw128_kmajor_desc(a_addr + koff), sw128_kmajor_desc(b_addr + koff), idesc,
+                                   m > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&tfull[b]);
+                    }
+                    if (ok) mma_commit(&empty[s]);
+                }
+            }
+            mma_commit(drain);          // all MMAs issued by this thread have finished
+            drain_wait(drain, 0);
+        }
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int ew = warp - 2;
+        const int quad = warp & 3;                // TMEM lanes 32*quad .. 32*quad+31
+        const int half = ew >> 2;                 // columns half*128 .. half*128+127 of the tile
+        const int row_in_tile = quad * 32 + lane;
+        uint32_t it = 0, kg = 0, tile = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++tile) {
+            int e, nb, mb;
+            decode_unit(u, nt, s_tstart, p.E, e, nb, mb);
+            const int row0 = s_off[e] + mb * kTileM;
+            const int cnt = min(kTileM, s_off[e + 1] - row0);
+            const bool warp_active = quad * 32 < cnt;
+            const bool row_ok = row_in_tile < cnt;
+            const int r = row0 + row_in_tile;
+
+            float acc[128];
+#pragma unroll
+            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+
+            for (int kb = 0; kb < KB && ok; ++kb, ++it) {
+                const int s = it % kStages;
+                float sa = 0.0f;
+                uint32_t sa4 = 0;
+                if (row_ok) {
+                    if (RECIPE == 0) sa = static_cast<const float*>(p.a_scale)[static_cast<size_t>(r) * KB + kb];
+                    else sa4 = static_cast<const uint32_t*>(p.a_scale)[static_cast<size_t>(r) * KB + kb];
+                }
+                // acquire the stage (its weight scales were written by the bulk copy)
+                if (!mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* ws_stage = smem + L::ws + s * kWsBytes + half * 128 * 4;
+                for (int g = 0; g < GPS; ++g, ++kg) {
+                    const int b = kg & 1;
+                    if (!mbar_wait(&tfull[b], (kg >> 1) & 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (warp_active) {
+                        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                               static_cast<uint32_t>(b * kTileN + half * 128);
+                        if (RECIPE == 0)
+                            promote_fp32(acc, taddr, reinterpret_cast<const float*>(ws_stage), sa);
+                        else
+                            promote_mx(acc, taddr, reinterpret_cast<const uint32_t*>(ws_stage),
+                                       static_cast<int>((sa4 >> (8 * g)) & 0xFFu), g);
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[b]);
+                }
+                if (!ok) break;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+            }
+            if (!ok) break;
+
+            if (MODE == 0) {
+                // ---- SwiGLU + requantization: acc[0:64] gate, acc[64:128] up, act columns c0..c0+63
+                const int I = p.N >> 1;
+                const int c0 = nb * 128 + half * 64;
+                if (warp_active) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) {
+                        float gt = acc[i], up = acc[64 + i];
+                        if (p.bias) {
+                            gt += __bfloat162float(p.bias[static_cast<size_t>(e) * p.N + c0 + i]);
+                            up += __bfloat162float(p.bias[static_cast<size_t>(e) * p.N + I + c0 + i]);
+                        }
+                        acc[i] = __fdiv_rn(gt, 1.0f + expf(-gt)) * up;
+                    }
+                }
+                if (RECIPE == 0) {
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(acc[i]));
+                    const int buf = tile & 1;
+                    s_amax[(buf * 2 + half) * 128 + row_in_tile] = amax;
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&amax_bar[buf]);
+                    if (!mbar_wait(&amax_bar[buf], (tile >> 1) & 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    amax = fmaxf(amax, s_amax[(buf * 2 + (half ^ 1)) * 128 + row_in_tile]);
+                    const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+                    if (warp_active && row_ok) {
+                        uint4* dst = reinterpret_cast<uint4*>(p.act_q + static_cast<size_t>(r) * I + c0);
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            uint4 q;
+                            q.x = e4m3x4(__fdiv_rn(acc[16 * w + 0], sc), __fdiv_rn(acc[16 * w + 1], sc),
+                                         __fdiv_rn(acc[16 * w + 2], sc), __fdiv_rn(acc[16 * w + 3], sc));
+                            q.y = e4m3x4(__fdiv_rn(acc[16 * w + 4], sc), __fdiv_rn(acc[16 * w + 5], sc),
+                                         __fdiv_rn(acc[16 * w + 6], sc), __fdiv_rn(acc[16 * w + 7], sc));
+                            q.z = e4m3x4(__fdiv_rn(acc[16 * w + 8], sc), __fdiv_rn(acc[16 * w + 9], sc),
+                                         __fdiv_rn(acc[16 * w + 10], sc), __fdiv_rn(acc[16 * w + 11], sc));
+                            q.w = e4m3x4(__fdiv_rn(acc[16 * w + 12], sc), __fdiv_rn(acc[16 * w + 13], sc),
+                                         __fdiv_rn(acc[16 * w + 14], sc), __fdiv_rn(acc[16 * w + 15], sc));
+                            dst[w] = q;
+                        }
+                        if (half == 0) static_cast<float*>(p.act_s)[static_cast<size_t>(r) * (I >> 7) + nb] = sc;
+                    }
+                } else if (warp_active && row_ok) {
+                    uint32_t* dst = reinterpret_cast<uint32_t*>(p.act_q + static_cast<size_t>(r) * I + c0);
+#pragma unroll
+                    for (int grp = 0; grp < 2; ++grp) {
+                        float amax = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(acc[32 * grp + i]));
+                        const int ex = mx_exponent(amax);
+                        const float inv = exp2_int(-ex);
+                        uint32_t q[8];
+#pragma unroll
+                        for (int w = 0; w < 8; ++w)
+                            q[w] = e4m3x4(acc[32 * grp + 4 * w] * inv, acc[32 * grp + 4 * w + 1] * inv,
+                                          acc[32 * grp + 4 * w + 2] * inv, acc[32 * grp + 4 * w + 3] * inv);
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + 8 * grp);
+                        d4[0] = make_uint4(q[0], q[1], q[2], q[3]);
+                        d4[1] = make_uint4(q[4], q[5], q[6], q[7]);
+                        static_cast<uint8_t*>(p.act_s)[static_cast<size_t>(r) * (I >> 5) + nb * 4 + half * 2 + grp] =
+                            static_cast<uint8_t>(ex + 127);
+                    }
+                }
+            } else {
+                // ---- down projection: + bias, fp32 rows
+                const int c0 = nb * kTileN + half * 128;
+                if (warp_active && row_ok && c0 < p.N) {
+                    float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.N + c0);
+#pragma unroll
+                    for (int c = 0; c < 128; c += 4) {
+                        float4 v = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                        if (p.bias) {
+                            const __nv_bfloat16* bb = p.bias + static_cast<size_t>(e) * p.N + c0 + c;
+                            v.x += __bfloat162float(bb[0]);
+                            v.y += __bfloat162float(bb[1]);
+                            v.z += __bfloat162float(bb[2]);
+                            v.w += __bfloat162float(bb[3]);
+                        }
+                        dst[c >> 2] = v;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+template <int MODE, int RECIPE>
+static cudaError_t launch_gemm_t(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
+                                 cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<MODE, RECIPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    k_grouped_gemm<MODE, RECIPE><<<num_sms, kThreads, kSmemBytes, s>>>(tmA, tmB, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
+                        cudaStream_t s) {
+    if (a.mode == 0) {
+        return a.recipe == 0 ? launch_gemm_t<0, 0>(a, tmA, tmB, num_sms, s)
+                             : launch_gemm_t<0, 1>(a, tmA, tmB, num_sms, s);
+    }
+    return a.recipe == 0 ? launch_gemm_t<1, 0>(a, tmA, tmB, num_sms, s) : launch_gemm_t<1, 1>(a, tmA, tmB, num_sms, s);
+}
+
+}  // namespace moe

@@ -1,0 +1,95 @@
+// moe_kernels.h -- host-side launchers of the kernels of libmoefp8.so (internal header).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kPermuteChunk = 1024;   // routed rows per histogram / scatter chunk
+constexpr int kTileM = 128;           // GEMM rows per tile
+constexpr int kTileN = 256;           // GEMM output columns per tile
+constexpr int kTileK = 128;           // K bytes (= E4M3 elements) per pipeline stage
+
+struct RouteArgs {
+    const float* logits;        // [T, E]
+    const float* pes;           // [E] or null
+    int32_t* idx;               // [T, K]
+    float* w;                   // [T, K]
+    int T, E, K, routing, renorm, G, kg, mode;
+    float rsf;
+};
+
+struct PermuteArgs {
+    const int32_t* idx;         // [A]
+    int32_t* hist;              // [chunks, E]  (per-chunk counts, then exclusive bases)
+    int32_t* counts;            // [E]
+    int32_t* offsets;           // [E + 1]
+    int32_t* tile_start;        // [E + 1]
+    int32_t* row_src;           // [A]
+    int32_t* row_of;            // [A]
+    int32_t* expert_counts;     // [E] or null (caller's copy)
+    int32_t* status;
+    int A, E, chunks;
+};
+
+struct QuantArgs {
+    const __nv_bfloat16* x;     // [T, H]
+    const int32_t* row_of;      // [T, K]
+    uint8_t* xq;                // [A, H]
+    void* xs;                   // [A, H/g]
+    int32_t* status;
+    int T, H, K, recipe;
+};
+
+struct CombineArgs {
+    const float* o;             // [A, H]
+    const int32_t* row_of;      // [T, K]
+    const float* w;             // [T, K]
+    __nv_bfloat16* y;           // [T, H]
+    int T, H, K;
+};
+
+struct TransformArgs {
+    const uint8_t* w13; const void* w13s; const uint8_t* w2; const void* w2s;
+    uint8_t* w13_t; void* w13s_t; uint8_t* w2_t; void* w2s_t;
+    int E, H, I, recipe;
+};
+
+struct GemmArgs {
+    int mode;                   // 0: gate+up, SwiGLU, requantize; 1: down projection
+    int recipe;
+    int N, K, E, A;
+    const int32_t* offsets;     // [E + 1]
+    const int32_t* tile_start;  // [E + 1]
+    const void* a_scale;        // [A, K/g]
+    const void* w_scale;        // recipe 0: fp32 [E, K/128, N]; recipe 1: u8 [E, K/128, N, 4]
+    const __nv_bfloat16* bias;  // [E, N] in the caller's column order, or null
+    uint8_t* act_q;             // mode 0: [A, N/2]
+    void* act_s;                // mode 0: [A, (N/2)/g]
+    float* out;                 // mode 1: [A, N]
+    int32_t* status;
+};
+
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s);
+cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                        int num_sms, cudaStream_t s);
+cudaError_t launch_selftest_wait(int32_t* status, uint32_t timeout_us, cudaStream_t s);
+
+// Column permutation applied to w13 by the transform: within each 256-column block nb,
+// [gate nb*128 + 0:64 | up nb*128 + 0:64 | gate nb*128 + 64:128 | up nb*128 + 64:128].
+// Returns the transformed row index of original column n (0 <= n < 2I).
+__host__ __device__ inline int w13_interleaved_row(int n, int I) {
+    const int is_up = n >= I;
+    const int i = is_up ? n - I : n;
+    const int nb = i >> 7, within = i & 127;
+    return nb * 256 + (within >> 6) * 128 + is_up * 64 + (within & 63);
+}
+
+}  // namespace moe

@@ -1,0 +1,441 @@
+// moefp8_api.cu -- the C ABI of libmoefp8.so (declared in include/moefp8.h): argument
+// validation before any launch, workspace layout, TMA descriptors, and the launch sequence of
+// the layer forward on the caller's stream.
+//
+// "metrale_model_layers fp8_grouped_tc_w8a8.rs": the step launches nothing unless the shapes
+// fit; "mlx_native ops/moe_gate.rs": every dimension > 0, top_k <= n_experts, buffer checks,
+// an InvalidArgument message; "MindIE-SD Fused MoE", routing selection: the grouped-routing
+// constraints; "MATE Mega MoE", Current Limits and Typical Flow.
+#include <cudaTypedefs.h>
+
+#include <array>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "moe_common.cuh"
+#include "moe_kernels.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int ok() {
+    g_err.clear();
+    return MOE_OK;
+}
+
+#define MOE_CUDA_TRY(expr)                                                                      \
+    do {                                                                                        \
+        cudaError_t _e = (expr);                                                                \
+        if (_e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(_e)); \
+    } while (0)
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int scale_group(const moe_config_t* c) { return c->recipe == 0 ? 128 : 32; }
+size_t scale_elem_bytes(const moe_config_t* c) { return c->recipe == 0 ? 4 : 1; }
+
+int check_config(const moe_config_t* c) {
+    if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
+    if (c->num_tokens <= 0) return fail(MOE_ERR_INVALID_ARG, "num_tokens must be > 0 (got %d)", c->num_tokens);
+    if (c->hidden <= 0) return fail(MOE_ERR_INVALID_ARG, "hidden must be > 0 (got %d)", c->hidden);
+    if (c->inter <= 0) return fail(MOE_ERR_INVALID_ARG, "inter must be > 0 (got %d)", c->inter);
+    if (c->num_experts <= 0) return fail(MOE_ERR_INVALID_ARG, "num_experts must be > 0 (got %d)", c->num_experts);
+    if (c->top_k < 1 || c->top_k > c->num_experts)
+        return fail(MOE_ERR_INVALID_ARG, "top_k (%d) must be in [1, num_experts=%d]", c->top_k, c->num_experts);
+    if (c->routing != 0 && c->routing != 1)
+        return fail(MOE_ERR_INVALID_ARG, "routing must be 0 (softmax) or 1 (sigmoid), got %d", c->routing);
+    if (c->recipe != 0 && c->recipe != 1)
+        return fail(MOE_ERR_INVALID_ARG, "recipe must be 0 (fp32 per 128) or 1 (MXFP8), got %d", c->recipe);
+    if (c->hidden % 128) return fail(MOE_ERR_UNSUPPORTED, "hidden (%d) must be a multiple of 128", c->hidden);
+    if (c->inter % 128) return fail(MOE_ERR_UNSUPPORTED, "inter (%d) must be a multiple of 128", c->inter);
+    if (c->num_experts > MOE_MAX_EXPERTS)
+        return fail(MOE_ERR_UNSUPPORTED, "num_experts (%d) exceeds %d", c->num_experts, MOE_MAX_EXPERTS);
+    if (c->group_count < 1 || c->num_experts % c->group_count)
+        return fail(MOE_ERR_UNSUPPORTED, "num_experts (%d) must be divisible by group_count (%d)", c->num_experts,
+                    c->group_count);
+    if (c->k_group < 1 || c->k_group > c->group_count)
+        return fail(MOE_ERR_UNSUPPORTED, "k_group (%d) must be in [1, group_count=%d]", c->k_group, c->group_count);
+    const int per_group = c->num_experts / c->group_count;
+    if (c->top_k > c->k_group * per_group)
+        return fail(MOE_ERR_UNSUPPORTED, "top_k (%d) exceeds the experts in the selected groups (%d)", c->top_k,
+                    c->k_group * per_group);
+    if (c->group_select_mode != 0 && c->group_select_mode != 1)
+        return fail(MOE_ERR_INVALID_ARG, "group_select_mode must be 0 or 1, got %d", c->group_select_mode);
+    if (c->group_select_mode == 1 && per_group < 2)
+        return fail(MOE_ERR_UNSUPPORTED, "group_select_mode 1 needs at least 2 experts per group");
+    const long long A = 1LL * c->num_tokens * c->top_k;
+    if (A > (1LL << 30) || 1LL * c->num_experts * 2 * c->inter > (1LL << 30) ||
+        1LL * c->num_experts * c->hidden > (1LL << 30))
+        return fail(MOE_ERR_UNSUPPORTED, "problem too large for 32-bit row indices");
+    return MOE_OK;
+}
+
+void layout_of(const moe_config_t* c, moe_workspace_layout_t* L) {
+    const size_t T = c->num_tokens, K = c->top_k, E = c->num_experts, H = c->hidden, I = c->inter;
+    const size_t A = T * K, g = scale_group(c), sb = scale_elem_bytes(c);
+    const size_t chunks = (A + moe::kPermuteChunk - 1) / moe::kPermuteChunk;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 1024);
+        return o;
+    };
+    L->status = take(16);
+    L->topk_idx = take(4 * A);
+    L->topk_weights = take(4 * A);
+    L->counts = take(4 * E);
+    L->offsets = take(4 * (E + 1));
+    L->tile_start = take(4 * (E + 1));
+    L->row_src = take(4 * A);
+    L->row_of = take(4 * A);
+    L->hist = take(4 * chunks * E);
+    L->xq = take(A * H);
+    L->xs = take(A * (H / g) * sb);
+    L->act_q = take(A * I);
+    L->act_s = take(A * (I / g) * sb);
+    L->o = take(4 * A * H);
+    L->total = off;
+}
+
+// ---- device facts, looked up once per device
+struct DeviceInfo {
+    int sms = 0;
+    int cc_major = 0, cc_minor = 0;
+};
+
+int device_info(DeviceInfo* out) {
+    static std::mutex mu;
+    static std::array<DeviceInfo, 64> cache{};
+    int dev = 0;
+    MOE_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev].sms == 0) {
+        DeviceInfo d;
+        MOE_CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+        MOE_CUDA_TRY(cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev));
+        MOE_CUDA_TRY(cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev));
+        cache[dev] = d;
+    }
+    *out = cache[dev];
+    if (out->cc_major != 10 || out->cc_minor != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "libmoefp8 is built for sm_100a (B200); device is sm_%d%d", out->cc_major,
+                    out->cc_minor);
+    return MOE_OK;
+}
+
+// ---- TMA descriptors (the driver entry point is fetched through the runtime; no -lcuda)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2D map over a row-major byte matrix [rows, cols] (cols = K, contiguous), box box_rows x 128,
+// 128-byte swizzle; rows past the end read as zero.
+int make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return MOE_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+// ============================================================================ profiler
+struct moe_profile {
+    std::vector<std::array<cudaEvent_t, MOE_NUM_STAGES + 1>> sets;
+    size_t used = 0;
+    double totals[MOE_NUM_STAGES] = {0};
+    int32_t calls = 0;
+};
+
+namespace {
+
+int prof_next(moe_profile* p, cudaEvent_t** ev) {
+    if (p->used == p->sets.size()) {
+        if (p->sets.size() >= 4096) return fail(MOE_ERR_INVALID_ARG, "profiler holds 4096 unread calls; read it");
+        std::array<cudaEvent_t, MOE_NUM_STAGES + 1> s{};
+        for (auto& e : s) MOE_CUDA_TRY(cudaEventCreate(&e));
+        p->sets.push_back(s);
+    }
+    *ev = p->sets[p->used++].data();
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_err.c_str(); }
+
+int moe_check_config(const moe_config_t* cfg) {
+    int rc = check_config(cfg);
+    return rc ? rc : ok();
+}
+
+int moe_transformed_weights_size(const moe_config_t* cfg, size_t* w13_bytes, size_t* w13s_bytes, size_t* w2_bytes,
+                                 size_t* w2s_bytes) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!w13_bytes || !w13s_bytes || !w2_bytes || !w2s_bytes) return fail(MOE_ERR_INVALID_ARG, "NULL size pointer");
+    const size_t E = cfg->num_experts, H = cfg->hidden, I = cfg->inter;
+    *w13_bytes = E * 2 * I * H;
+    *w13s_bytes = E * (H / 128) * 2 * I * 4;
+    *w2_bytes = E * H * I;
+    *w2s_bytes = E * (I / 128) * H * 4;
+    return ok();
+}
+
+int moe_transform_weights(const moe_config_t* cfg, const void* w13, const void* w13_scale, const void* w2,
+                          const void* w2_scale, void* w13_t, void* w13s_t, void* w2_t, void* w2s_t, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!w13 || !w13_scale || !w2 || !w2_scale || !w13_t || !w13s_t || !w2_t || !w2s_t)
+        return fail(MOE_ERR_INVALID_ARG, "moe_transform_weights: NULL pointer");
+    if (!aligned(w13_scale, 4) || !aligned(w2_scale, 4) || !aligned(w13s_t, 16) || !aligned(w2s_t, 16) ||
+        !aligned(w13_t, 16) || !aligned(w2_t, 16))
+        return fail(MOE_ERR_INVALID_ARG, "moe_transform_weights: misaligned buffer (outputs need 16 bytes)");
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    moe::TransformArgs a{static_cast<const uint8_t*>(w13), w13_scale, static_cast<const uint8_t*>(w2), w2_scale,
+                         static_cast<uint8_t*>(w13_t), w13s_t, static_cast<uint8_t*>(w2_t), w2s_t,
+                         cfg->num_experts, cfg->hidden, cfg->inter, cfg->recipe};
+    MOE_CUDA_TRY(moe::launch_transform(a, static_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+int moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!bytes) return fail(MOE_ERR_INVALID_ARG, "NULL bytes pointer");
+    moe_workspace_layout_t L;
+    layout_of(cfg, &L);
+    *bytes = L.total;
+    return ok();
+}
+
+int moe_workspace_layout(const moe_config_t* cfg, moe_workspace_layout_t* layout) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!layout) return fail(MOE_ERR_INVALID_ARG, "NULL layout pointer");
+    layout_of(cfg, layout);
+    return ok();
+}
+
+int moe_route(const moe_config_t* cfg, const float* router_logits, const float* per_expert_scale, int32_t* topk_idx,
+              float* topk_weights, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!router_logits || !topk_idx || !topk_weights) return fail(MOE_ERR_INVALID_ARG, "moe_route: NULL pointer");
+    if (!aligned(router_logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_weights, 4))
+        return fail(MOE_ERR_INVALID_ARG, "moe_route: misaligned buffer");
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    moe::RouteArgs a{router_logits, per_expert_scale, topk_idx, topk_weights, cfg->num_tokens, cfg->num_experts,
+                     cfg->top_k, cfg->routing, cfg->renormalize, cfg->group_count, cfg->k_group,
+                     cfg->group_select_mode, cfg->routed_scaling_factor};
+    MOE_CUDA_TRY(moe::launch_route(a, static_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, const float* router_logits,
+                         const float* per_expert_scale, const int32_t* topk_idx, const float* topk_weights,
+                         const void* w13_t, const void* w13s_t, const void* w2_t, const void* w2s_t,
+                         const void* w13_bias, const void* w2_bias, void* y, int32_t* expert_counts, void* workspace,
+                         size_t workspace_bytes, moe_profile_t* prof, void* stream_) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!hidden_states || !y || !w13_t || !w13s_t || !w2_t || !w2s_t || !workspace)
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
+    if ((router_logits == nullptr) == (topk_idx == nullptr))
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward: pass exactly one of router_logits and topk_idx");
+    if (topk_idx && !topk_weights) return fail(MOE_ERR_INVALID_ARG, "moe_forward: topk_idx needs topk_weights");
+    if (!aligned(hidden_states, 16) || !aligned(y, 16) || !aligned(w13_t, 16) || !aligned(w2_t, 16) ||
+        !aligned(w13s_t, 16) || !aligned(w2s_t, 16) || !aligned(workspace, 256) ||
+        (router_logits && !aligned(router_logits, 4)) || (topk_idx && !aligned(topk_idx, 4)) ||
+        (topk_weights && !aligned(topk_weights, 4)) || (w13_bias && !aligned(w13_bias, 2)) ||
+        (w2_bias && !aligned(w2_bias, 2)) || (expert_counts && !aligned(expert_counts, 4)))
+        return fail(MOE_ERR_INVALID_ARG,
+                    "moe_forward: misaligned buffer (hidden_states, y and weights need 16 bytes, workspace 256)");
+    moe_workspace_layout_t L;
+    layout_of(cfg, &L);
+    if (workspace_bytes < L.total)
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward: workspace has %zu bytes, needs %zu", workspace_bytes, L.total);
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+
+    const int T = cfg->num_tokens, K = cfg->top_k, E = cfg->num_experts, H = cfg->hidden, I = cfg->inter;
+    const int A = T * K;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
+    int32_t* status = static_cast<int32_t*>(at(L.status));
+    const int32_t* idx = topk_idx ? topk_idx : static_cast<const int32_t*>(at(L.topk_idx));
+    const float* wts = topk_idx ? topk_weights : static_cast<const float*>(at(L.topk_weights));
+
+    CUtensorMap tm_x, tm_w13, tm_act, tm_w2;
+    if ((rc = make_kmajor_map(&tm_x, at(L.xq), A, H, moe::kTileM))) return rc;
+    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(E) * 2 * I, H, moe::kTileN))) return rc;
+    if ((rc = make_kmajor_map(&tm_act, at(L.act_q), A, I, moe::kTileM))) return rc;
+    if ((rc = make_kmajor_map(&tm_w2, w2_t, static_cast<uint64_t>(E) * H, I, moe::kTileN))) return rc;
+
+    cudaEvent_t* ev = nullptr;
+    if (prof && (rc = prof_next(prof, &ev))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream_);
+    auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], s) : cudaSuccess; };
+
+    MOE_CUDA_TRY(mark(0));
+    MOE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    if (router_logits) {
+        moe::RouteArgs ra{router_logits, per_expert_scale, static_cast<int32_t*>(at(L.topk_idx)),
+                          static_cast<float*>(at(L.topk_weights)), T, E, K, cfg->routing, cfg->renormalize,
+                          cfg->group_count, cfg->k_group, cfg->group_select_mode, cfg->routed_scaling_factor};
+        MOE_CUDA_TRY(moe::launch_route(ra, s));
+    }
+    MOE_CUDA_TRY(mark(1));
+    moe::PermuteArgs pa{idx, static_cast<int32_t*>(at(L.hist)), static_cast<int32_t*>(at(L.counts)),
+                        static_cast<int32_t*>(at(L.offsets)), static_cast<int32_t*>(at(L.tile_start)),
+                        static_cast<int32_t*>(at(L.row_src)), static_cast<int32_t*>(at(L.row_of)), expert_counts,
+                        status, A, E, (A + moe::kPermuteChunk - 1) / moe::kPermuteChunk};
+    MOE_CUDA_TRY(moe::launch_permute(pa, s));
+    MOE_CUDA_TRY(mark(2));
+    moe::QuantArgs qa{static_cast<const __nv_bfloat16*>(hidden_states), static_cast<const int32_t*>(at(L.row_of)),
+                      static_cast<uint8_t*>(at(L.xq)), at(L.xs), status, T, H, K, cfg->recipe};
+    MOE_CUDA_TRY(moe::launch_quant(qa, s));
+    MOE_CUDA_TRY(mark(3));
+    moe::GemmArgs g1{};
+    g1.mode = 0;
+    g1.recipe = cfg->recipe;
+    g1.N = 2 * I;
+    g1.K = H;
+    g1.E = E;
+    g1.A = A;
+    g1.offsets = static_cast<const int32_t*>(at(L.offsets));
+    g1.tile_start = static_cast<const int32_t*>(at(L.tile_start));
+    g1.a_scale = at(L.xs);
+    g1.w_scale = w13s_t;
+    g1.bias = static_cast<const __nv_bfloat16*>(w13_bias);
+    g1.act_q = static_cast<uint8_t*>(at(L.act_q));
+    g1.act_s = at(L.act_s);
+    g1.status = status;
+    MOE_CUDA_TRY(moe::launch_gemm(g1, tm_x, tm_w13, di.sms, s));
+    MOE_CUDA_TRY(mark(4));
+    moe::GemmArgs g2 = g1;
+    g2.mode = 1;
+    g2.N = H;
+    g2.K = I;
+    g2.a_scale = at(L.act_s);
+    g2.w_scale = w2s_t;
+    g2.bias = static_cast<const __nv_bfloat16*>(w2_bias);
+    g2.act_q = nullptr;
+    g2.act_s = nullptr;
+    g2.out = static_cast<float*>(at(L.o));
+    MOE_CUDA_TRY(moe::launch_gemm(g2, tm_act, tm_w2, di.sms, s));
+    MOE_CUDA_TRY(mark(5));
+    moe::CombineArgs ca{static_cast<const float*>(at(L.o)), static_cast<const int32_t*>(at(L.row_of)), wts,
+                        static_cast<__nv_bfloat16*>(y), T, H, K};
+    MOE_CUDA_TRY(moe::launch_combine(ca, s));
+    MOE_CUDA_TRY(mark(6));
+    return ok();
+}
+
+int moe_forward(const moe_config_t* cfg, const void* hidden_states, const float* router_logits,
+                const float* per_expert_scale, const int32_t* topk_idx, const float* topk_weights, const void* w13_t,
+                const void* w13s_t, const void* w2_t, const void* w2s_t, const void* w13_bias, const void* w2_bias,
+                void* y, int32_t* expert_counts, void* workspace, size_t workspace_bytes, void* stream) {
+    return moe_forward_profiled(cfg, hidden_states, router_logits, per_expert_scale, topk_idx, topk_weights, w13_t,
+                                w13s_t, w2_t, w2s_t, w13_bias, w2_bias, y, expert_counts, workspace, workspace_bytes,
+                                nullptr, stream);
+}
+
+int moe_profile_create(moe_profile_t** prof) {
+    if (!prof) return fail(MOE_ERR_INVALID_ARG, "NULL profiler pointer");
+    *prof = new moe_profile();
+    return ok();
+}
+
+int moe_profile_destroy(moe_profile_t* prof) {
+    if (!prof) return ok();
+    for (auto& s : prof->sets)
+        for (auto& e : s) cudaEventDestroy(e);
+    delete prof;
+    return ok();
+}
+
+int moe_profile_read(moe_profile_t* prof, float* stage_ms, int32_t* calls) {
+    if (!prof) return fail(MOE_ERR_INVALID_ARG, "NULL profiler");
+    for (size_t i = 0; i < prof->used; ++i) {
+        auto& s = prof->sets[i];
+        MOE_CUDA_TRY(cudaEventSynchronize(s[MOE_NUM_STAGES]));
+        for (int k = 0; k < MOE_NUM_STAGES; ++k) {
+            float ms = 0.f;
+            MOE_CUDA_TRY(cudaEventElapsedTime(&ms, s[k], s[k + 1]));
+            prof->totals[k] += ms;
+        }
+        prof->calls++;
+    }
+    prof->used = 0;
+    if (stage_ms)
+        for (int k = 0; k < MOE_NUM_STAGES; ++k) stage_ms[k] = static_cast<float>(prof->totals[k]);
+    if (calls) *calls = prof->calls;
+    return ok();
+}
+
+int moe_profile_reset(moe_profile_t* prof) {
+    if (!prof) return fail(MOE_ERR_INVALID_ARG, "NULL profiler");
+    prof->used = 0;
+    prof->calls = 0;
+    for (double& t : prof->totals) t = 0;
+    return ok();
+}
+
+int moe_read_status(const void* workspace, int32_t* status, void* stream) {
+    if (!workspace || !status) return fail(MOE_ERR_INVALID_ARG, "moe_read_status: NULL pointer");
+    MOE_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    MOE_CUDA_TRY(cudaMemcpy(status, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost));
+    return ok();
+}
+
+int moe_selftest_bounded_wait(int32_t* status, uint32_t timeout_us, void* stream) {
+    if (!status) return fail(MOE_ERR_INVALID_ARG, "moe_selftest_bounded_wait: NULL status");
+    if (timeout_us == 0 || timeout_us > 10000000u)
+        return fail(MOE_ERR_INVALID_ARG, "timeout_us must be in [1, 10000000]");
+    DeviceInfo di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    MOE_CUDA_TRY(moe::launch_selftest_wait(status, timeout_us, static_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+}  // extern "C"

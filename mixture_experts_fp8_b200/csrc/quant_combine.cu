@@ -1,0 +1,191 @@
+// quant_combine.cu -- the two HBM-bound ends of the layer.
+//
+// k_quant (dispatch side): dynamic E4M3 quantization of the layer input, scattered straight
+// into expert-contiguous order.  "metrale_model_layers fp8_grouped_tc_w8a8.rs", module doc:
+// the layer input is quantized to E4M3 per (row, 128 group); "DeepGEMM PR #371", Changes:
+// UE8M0 scale factors per 32 elements.  Each token is quantized once and its codes are
+// written to the k permuted rows it was routed to (the codes do not depend on the expert).
+//   recipe 0: s = amax / 448 (IEEE division), q = e4m3_rn_satfinite(x / s); amax 0 -> s = 1
+//   recipe 1: s = 2^e, e the smallest with amax <= 448 * 2^e; byte e + 127; q = e4m3(x * 2^-e)
+//
+// k_combine: y[t] = bf16_rn( sum_j w[t,j] * o[row_of[t,j]] ), fp32, fixed slot order, no
+// atomics ("MindIE-SD Fused MoE", execution flow: combine; "MATE Mega MoE", Current Limits:
+// contiguous bf16 output).
+#include "moe_common.cuh"
+#include "moe_kernels.h"
+
+namespace moe {
+
+// One warp per (token, 128-column block).  Lane l owns columns 4l .. 4l+3 of the block.
+__global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
+    const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int nblk = a.H >> 7;
+    if (gw >= a.T * nblk) return;
+    const int t = gw / nblk, cb = gw - t * nblk;
+    const uint2 raw = *reinterpret_cast<const uint2*>(a.x + static_cast<size_t>(t) * a.H + cb * 128 + 4 * lane);
+    const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+    const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+    const float v0 = __low2float(p0), v1 = __high2float(p0), v2 = __low2float(p1), v3 = __high2float(p1);
+    float amax = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
+    uint32_t q;
+    float s32 = 1.0f;
+    uint8_t e8 = 127;
+    if (a.recipe == 0) {
+        amax = warp_max(amax);
+        s32 = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        q = e4m3x4(__fdiv_rn(v0, s32), __fdiv_rn(v1, s32), __fdiv_rn(v2, s32), __fdiv_rn(v3, s32));
+    } else {
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const int e = mx_exponent(amax);
+        const float inv = exp2_int(-e);                 // x * 2^-e == x / 2^e exactly
+        q = e4m3x4(v0 * inv, v1 * inv, v2 * inv, v3 * inv);
+        e8 = static_cast<uint8_t>(e + 127);
+    }
+    const int A = a.T * a.K;
+    for (int j = 0; j < a.K; ++j) {
+        const int r = a.row_of[static_cast<size_t>(t) * a.K + j];
+        if (r < 0 || r >= A) {
+            if (lane == 0) set_status(a.status, MOE_ERR_BOUNDS);
+            continue;
+        }
+        *reinterpret_cast<uint32_t*>(a.xq + static_cast<size_t>(r) * a.H + cb * 128 + 4 * lane) = q;
+        if (a.recipe == 0) {
+            if (lane == 0) static_cast<float*>(a.xs)[static_cast<size_t>(r) * nblk + cb] = s32;
+        } else if ((lane & 7) == 0) {
+            static_cast<uint8_t*>(a.xs)[static_cast<size_t>(r) * (a.H >> 5) + cb * 4 + (lane >> 3)] = e8;
+        }
+    }
+}
+
+cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s) {
+    const int warps = a.T * (a.H >> 7);
+    k_quant<<<(warps + 7) / 8, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+// One block per token; thread i handles float4 columns i, i + 256, ...
+__global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
+    __shared__ int s_row[MOE_MAX_EXPERTS];
+    __shared__ float s_w[MOE_MAX_EXPERTS];
+    const int t = blockIdx.x;
+    const int A = a.T * a.K;
+    for (int j = threadIdx.x; j < a.K; j += blockDim.x) {
+        int r = a.row_of[static_cast<size_t>(t) * a.K + j];
+        s_row[j] = (r >= 0 && r < A) ? r : 0;
+        s_w[j] = a.w[static_cast<size_t>(t) * a.K + j];
+    }
+    __syncthreads();
+    const int H4 = a.H >> 2;
+    for (int c = threadIdx.x; c < H4; c += blockDim.x) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < a.K; ++j) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(a.o + static_cast<size_t>(s_row[j]) * a.H) + c);
+            const float w = s_w[j];
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 out;
+        out.x = *reinterpret_cast<uint32_t*>(&lo);
+        out.y = *reinterpret_cast<uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(a.y + static_cast<size_t>(t) * a.H)[c] = out;
+    }
+}
+
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
+    k_combine<<<a.T, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// Weight transform (offline): E4M3 codes [E, K, N] -> K-major [E, N', K], with w13's columns
+// interleaved (moe::w13_interleaved_row), and the block scales re-laid to match:
+//   recipe 0: fp32 [E, K/128, N] -> [E, K/128, N'] (columns permuted like the codes)
+//   recipe 1: UE8M0 [E, K/32, N] -> [E, K/128, N', 4] (the four 32-deep blocks of each 128-deep
+//             stage packed into one 32-bit word per column)
+// ("MATE Mega MoE", transform_weights_for_mega_moe; "DeepGEMM PR #371", 4-packed UE8M0.)
+__global__ void __launch_bounds__(256) k_transpose_codes(const uint8_t* src, uint8_t* dst, int K,
+                                                        int N, int interleave_I) {
+    __shared__ uint8_t tile[64][65];
+    const int e = blockIdx.z;
+    const int k0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+    const uint8_t* s = src + static_cast<size_t>(e) * K * N;
+    uint8_t* d = dst + static_cast<size_t>(e) * K * N;
+    for (int i = threadIdx.x; i < 64 * 64; i += 256) {
+        const int kk = i / 64, nn = i % 64;
+        if (k0 + kk < K && n0 + nn < N) tile[kk][nn] = s[static_cast<size_t>(k0 + kk) * N + n0 + nn];
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 64 * 64; i += 256) {
+        const int nn = i / 64, kk = i % 64;
+        const int n = n0 + nn, k = k0 + kk;
+        if (n < N && k < K) {
+            const int row = interleave_I ? w13_interleaved_row(n, interleave_I) : n;
+            d[static_cast<size_t>(row) * K + k] = tile[kk][nn];
+        }
+    }
+}
+
+__global__ void k_transform_scales(const void* src, void* dst, int E, int K, int N, int recipe,
+                                   int interleave_I) {
+    const size_t total = static_cast<size_t>(E) * (K / 128) * N;
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const int n = static_cast<int>(i % N);
+        const size_t ek = i / N;                        // e * (K/128) + kb
+        const int row = interleave_I ? w13_interleaved_row(n, interleave_I) : n;
+        const size_t o = ek * N + row;
+        if (recipe == 0) {
+            static_cast<float*>(dst)[o] = static_cast<const float*>(src)[ek * N + n];
+        } else {
+            const size_t e = ek / (K / 128), kb = ek % (K / 128);
+            const uint8_t* s = static_cast<const uint8_t*>(src) + (e * (K / 32) + kb * 4) * N + n;
+            uint32_t w = static_cast<uint32_t>(s[0]) | (static_cast<uint32_t>(s[N]) << 8) |
+                         (static_cast<uint32_t>(s[2 * static_cast<size_t>(N)]) << 16) |
+                         (static_cast<uint32_t>(s[3 * static_cast<size_t>(N)]) << 24);
+            static_cast<uint32_t*>(dst)[o] = w;
+        }
+    }
+}
+
+cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s) {
+    const int H = a.H, I = a.I, E = a.E;
+    k_transpose_codes<<<dim3((2 * I + 63) / 64, (H + 63) / 64, E), 256, 0, s>>>(a.w13, a.w13_t, H, 2 * I, I);
+    k_transpose_codes<<<dim3((H + 63) / 64, (I + 63) / 64, E), 256, 0, s>>>(a.w2, a.w2_t, I, H, 0);
+    k_transform_scales<<<1024, 256, 0, s>>>(a.w13s, a.w13s_t, E, H, 2 * I, a.recipe, I);
+    k_transform_scales<<<1024, 256, 0, s>>>(a.w2s, a.w2s_t, E, I, H, a.recipe, 0);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// Failure-detection self test: wait on an mbarrier that nothing completes, bounded by
+// timeout_us, then record MOE_ERR_TIMEOUT and return.
+__global__ void k_selftest_wait(int32_t* status, uint32_t timeout_us) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t a = smem_u32(&bar);
+        const unsigned long long t0 = globaltimer_ns();
+        bool done = false;
+        while (!(done = mbar_try_wait(a, 0))) {
+            if (globaltimer_ns() - t0 > 1000ull * timeout_us) break;
+        }
+        *status = done ? MOE_OK : MOE_ERR_TIMEOUT;
+    }
+}
+
+cudaError_t launch_selftest_wait(int32_t* status, uint32_t timeout_us, cudaStream_t s) {
+    k_selftest_wait<<<1, 32, 0, s>>>(status, timeout_us);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,94 @@
+"""The C ABI library on a machine without a GPU: it loads, exports every entry point that
+include/moefp8.h declares, and validates arguments before touching the device (errors carry a
+message; "mlx_native ops/moe_gate.rs" validation and "MindIE-SD Fused MoE" constraints)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_fp8_b200 as moe
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "moefp8.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(moe.EXPORTED)
+
+
+def test_config_struct_layout():
+    assert ctypes.sizeof(moe._Cfg) == 48
+
+
+def cfg(**kw):
+    base = dict(num_tokens=16, hidden=256, inter=256, num_experts=8, top_k=2)
+    base.update(kw)
+    return moe.Config(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_tokens=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(hidden=-128), moe.MOE_ERR_INVALID_ARG),
+    (dict(top_k=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(top_k=9), moe.MOE_ERR_INVALID_ARG),
+    (dict(routing=2), moe.MOE_ERR_INVALID_ARG),
+    (dict(recipe=3), moe.MOE_ERR_INVALID_ARG),
+    (dict(hidden=200), moe.MOE_ERR_UNSUPPORTED),
+    (dict(inter=192), moe.MOE_ERR_UNSUPPORTED),
+    (dict(num_experts=512, top_k=2), moe.MOE_ERR_UNSUPPORTED),
+    (dict(group_count=3), moe.MOE_ERR_UNSUPPORTED),
+    (dict(group_count=4, k_group=5), moe.MOE_ERR_UNSUPPORTED),
+    (dict(group_count=4, k_group=1, top_k=3), moe.MOE_ERR_UNSUPPORTED),
+    (dict(group_count=8, group_select_mode=1), moe.MOE_ERR_UNSUPPORTED),
+])
+def test_validation(kw, code):
+    with pytest.raises(moe.MoeError) as e:
+        moe.check_config(cfg(**kw))
+    assert e.value.code == code
+    assert len(str(e.value)) > 10
+
+
+def test_valid_configs_and_sizes():
+    import synth
+    for name, s in synth.SHAPES.items():
+        c = moe.Config(**s.cfg())
+        moe.check_config(c)
+        lay = moe.workspace_layout(c)
+        assert lay["total"] == moe.workspace_size(c)
+        A = s.num_tokens * s.top_k
+        assert lay["o"] + 4 * A * s.hidden <= lay["total"]
+        assert all(v % 1024 == 0 for k, v in lay.items() if k != "total")
+        w13, w13s, w2, w2s = moe.transformed_weights_size(c)
+        assert w13 == s.num_experts * s.hidden * 2 * s.inter and w2 == s.num_experts * s.inter * s.hidden
+        assert w13s == s.num_experts * (s.hidden // 128) * 2 * s.inter * 4
+
+
+def test_forward_rejects_bad_pointers_before_any_cuda_call():
+    lib = moe.lib()
+    c = cfg().c()
+    rc = lib.moe_forward(ctypes.byref(c), None, None, None, None, None, None, None, None, None,
+                         None, None, None, None, None, 0, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+    assert b"NULL" in lib.moe_last_error()
+
+
+def test_interleave_is_a_permutation():
+    # mirror of the transform's column order, checked for bijectivity
+    I = 384
+    def row(n):
+        up = n >= I
+        i = n - I if up else n
+        return (i >> 7) * 256 + ((i & 127) >> 6) * 128 + up * 64 + (i & 63)
+    rows = sorted(row(n) for n in range(2 * I))
+    assert rows == list(range(2 * I))
