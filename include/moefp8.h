@@ -76,8 +76,10 @@ typedef struct {
 } moe_config_t;
 
 /* Byte offsets of the regions inside a forward workspace (for tests and diagnostics).
- * A = num_tokens * top_k routed rows; g = 128 (recipe 0) or 32 (recipe 1); scales are fp32
- * (recipe 0) or UE8M0 bytes (recipe 1).  All offsets are multiples of 1024. */
+ * A = num_tokens * top_k routed rows.  Scales are stored K-block-major: one 4-byte word per
+ * (128-column block, row) with a row stride of scale_rows words; the word is the fp32 scale
+ * (recipe 0) or the four UE8M0 bytes of the block's four 32-column groups, lowest group in the
+ * lowest byte (recipe 1).  All offsets are multiples of 1024. */
 typedef struct {
     size_t status;       /* int32 status word (MOE_OK or a device MOE_ERR_*)             */
     size_t topk_idx;     /* int32 [T, k]   routing computed by moe_forward               */
@@ -89,10 +91,11 @@ typedef struct {
     size_t row_of;       /* int32 [T, k]   permuted row of routed row (t, j)             */
     size_t hist;         /* int32 [chunks, E] per-chunk expert histograms                */
     size_t xq;           /* E4M3  [A, H]   quantized activations in permuted order       */
-    size_t xs;           /* scale [A, H/g]                                               */
+    size_t xs;           /* word  [H/128, scale_rows]                                    */
     size_t act_q;        /* E4M3  [A, I]   requantized SwiGLU products                   */
-    size_t act_s;        /* scale [A, I/g]                                               */
+    size_t act_s;        /* word  [I/128, scale_rows]                                    */
     size_t o;            /* fp32  [A, H]   down-projection output per permuted row       */
+    size_t scale_rows;   /* row stride (in words) of xs and act_s; >= A                  */
     size_t total;        /* bytes the workspace needs                                    */
 } moe_workspace_layout_t;
 
@@ -155,8 +158,8 @@ int moe_route(const moe_config_t *cfg, const float *router_logits, const float *
  *                                           router_logits and topk_idx must be non-NULL.
  *                                           The k ids of a token must be distinct, in [0, E).
  *   w13_t .. w2s_t    device, from moe_transform_weights with the same cfg fields
- *   w13_bias          device bf16 [E, 2I] or NULL
- *   w2_bias           device bf16 [E, H] or NULL
+ *   w13_bias          device bf16 [E, 2I] or NULL (16-byte aligned)
+ *   w2_bias           device bf16 [E, H] or NULL (16-byte aligned)
  *   y                 device bf16 [T, H], contiguous; out
  *   expert_counts     device int32 [E] or NULL; out: rows routed to each expert
  *   workspace         device, >= moe_workspace_size bytes, 1024-byte aligned; scratch owned by

@@ -51,7 +51,8 @@ class _Cfg(ctypes.Structure):
 
 
 _LAYOUT_FIELDS = ("status", "topk_idx", "topk_weights", "counts", "offsets", "tile_start",
-                  "row_src", "row_of", "hist", "xq", "xs", "act_q", "act_s", "o", "total")
+                  "row_src", "row_of", "hist", "xq", "xs", "act_q", "act_s", "o", "scale_rows",
+                  "total")
 
 
 class _Layout(ctypes.Structure):

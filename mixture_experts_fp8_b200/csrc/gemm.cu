@@ -9,13 +9,15 @@
 // quantized SiLU products, then the down projection; "MATE Mega MoE", API: swiglu;
 // "MindIE-SD Fused MoE", parameter table: w13_bias / w2_bias.
 //
-// Design (one persistent CTA per SM, 320 threads):
+// Design (one persistent CTA per SM, 384 threads = three warpgroups):
 //   warp 0   TMA producer: per 128-deep K stage, a 128x128 A tile and a 256x128 B tile (both
 //            K-major, 128-byte swizzle) plus the 256 weight scales of the stage (bulk copy).
 //   warp 1   MMA issuer (one thread): tcgen05.mma.kind::f8f6f4, M=128 N=256 K=32.  Each scale
 //            group (128 deep for recipe 0, 32 for recipe 1) is accumulated alone into one of two
 //            256-column fp32 TMEM buffers.
-//   warps 2-9 epilogue: a warp reads its 32 TMEM lanes (= tile rows), half of the columns each;
+//   warps 2-3 idle.  Warpgroup 0 gives registers back (setmaxnreg.dec to 40).
+//   warps 4-11 epilogue (setmaxnreg.inc to 232): a warp reads its 32 TMEM lanes (= tile rows),
+//            half of the columns each;
 //            every group partial is multiplied by a_s * w_s and added into fp32 registers (the
 //            "promotion"), then the tile's epilogue runs from registers.
 // Work unit = (expert, 256-column block, 128-row block), enumerated expert by expert, column
@@ -31,19 +33,24 @@ namespace moe {
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kEpiWarps = 8;
+constexpr int kFirstEpiWarp = 4;
+constexpr int kRegsLow = 40, kRegsHigh = 232;      // 128 * 40 + 256 * 232 = 384 * 168 (65536 / 384 -> 168)
 constexpr uint32_t kABytes = kTileM * kTileK;      // 16 KB
 constexpr uint32_t kBBytes = kTileN * kTileK;      // 32 KB
-constexpr uint32_t kWsBytes = kTileN * 4;          // fp32 or 4 x UE8M0 per column
+constexpr uint32_t kWsBytes = kTileN * 4;          // weight scales: fp32 or 4 x UE8M0 per column
+constexpr uint32_t kSaWords = kTileM + 4;          // activation scales of the tile's rows (+ 16-byte alignment)
+constexpr uint32_t kSaBytes = kSaWords * 4;
+constexpr uint32_t kScaleSlot = 2048;              // per stage: [weight scales | activation scales]
 constexpr uint32_t kTmemCols = 2 * kTileN;         // two fp32 accumulators
 constexpr unsigned long long kDrainLimitNs = 100000000ull;
 
 struct L {
     static constexpr uint32_t a = 0;
     static constexpr uint32_t b = a + kStages * kABytes;
-    static constexpr uint32_t ws = b + kStages * kBBytes;
-    static constexpr uint32_t bars = ws + kStages * kWsBytes;
+    static constexpr uint32_t sc = b + kStages * kBBytes;
+    static constexpr uint32_t bars = sc + kStages * kScaleSlot;
     static constexpr uint32_t nbars = 2 * kStages + 7;   // full, empty, tfull[2], tempty[2], drain, amax[2]
     static constexpr uint32_t misc = bars + nbars * 8;   // tmem holder, abort flag
     static constexpr uint32_t amax = misc + 16;          // float [2 buffers][2 halves][128 rows]
@@ -78,20 +85,31 @@ __device__ __forceinline__ void decode_unit(int u, int nt, const int* tstart, in
     mb = local - nb * mt;
 }
 
-// acc[j] += P[j] * (sa * ws[j]) for the 128 columns of this thread's half.
+// acc[j] += P[j] * (sa * ws[j]) for the 128 columns of this thread's half: two rounds of two
+// 32-column TMEM loads, one wait each.
 __device__ __forceinline__ void promote_fp32(float (&acc)[128], uint32_t taddr, const float* ws, float sa) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint32_t v[16];
-        MOE_TMEM_LD16(taddr + c * 16, v);
-        MOE_TMEM_WAIT_LD16(v);
+    for (int c = 0; c < 2; ++c) {
+        uint32_t v[32], u[32];
+        MOE_TMEM_LD32(taddr + c * 64, v);
+        MOE_TMEM_LD32(taddr + c * 64 + 32, u);
+        MOE_TMEM_WAIT_LD(v);
+        MOE_TMEM_WAIT_LD(u);
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-            const float4 w4 = *reinterpret_cast<const float4*>(ws + c * 16 + j);
-            acc[c * 16 + j + 0] = fmaf(__uint_as_float(v[j + 0]), sa * w4.x, acc[c * 16 + j + 0]);
-            acc[c * 16 + j + 1] = fmaf(__uint_as_float(v[j + 1]), sa * w4.y, acc[c * 16 + j + 1]);
-            acc[c * 16 + j + 2] = fmaf(__uint_as_float(v[j + 2]), sa * w4.z, acc[c * 16 + j + 2]);
-            acc[c * 16 + j + 3] = fmaf(__uint_as_float(v[j + 3]), sa * w4.w, acc[c * 16 + j + 3]);
+        for (int j = 0; j < 32; j += 4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(ws + c * 64 + j);
+            acc[c * 64 + j + 0] = fmaf(__uint_as_float(v[j + 0]), sa * w4.x, acc[c * 64 + j + 0]);
+            acc[c * 64 + j + 1] = fmaf(__uint_as_float(v[j + 1]), sa * w4.y, acc[c * 64 + j + 1]);
+            acc[c * 64 + j + 2] = fmaf(__uint_as_float(v[j + 2]), sa * w4.z, acc[c * 64 + j + 2]);
+            acc[c * 64 + j + 3] = fmaf(__uint_as_float(v[j + 3]), sa * w4.w, acc[c * 64 + j + 3]);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(ws + c * 64 + 32 + j);
+            acc[c * 64 + 32 + j + 0] = fmaf(__uint_as_float(u[j + 0]), sa * w4.x, acc[c * 64 + 32 + j + 0]);
+            acc[c * 64 + 32 + j + 1] = fmaf(__uint_as_float(u[j + 1]), sa * w4.y, acc[c * 64 + 32 + j + 1]);
+            acc[c * 64 + 32 + j + 2] = fmaf(__uint_as_float(u[j + 2]), sa * w4.z, acc[c * 64 + 32 + j + 2]);
+            acc[c * 64 + 32 + j + 3] = fmaf(__uint_as_float(u[j + 3]), sa * w4.w, acc[c * 64 + 32 + j + 3]);
         }
     }
 }
@@ -100,14 +118,21 @@ __device__ __forceinline__ void promote_fp32(float (&acc)[128], uint32_t taddr, 
 __device__ __forceinline__ void promote_mx(float (&acc)[128], uint32_t taddr, const uint32_t* ws4, int ea,
                                            int g) {
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint32_t v[16];
-        MOE_TMEM_LD16(taddr + c * 16, v);
-        MOE_TMEM_WAIT_LD16(v);
+    for (int c = 0; c < 2; ++c) {
+        uint32_t v[32], u[32];
+        MOE_TMEM_LD32(taddr + c * 64, v);
+        MOE_TMEM_LD32(taddr + c * 64 + 32, u);
+        MOE_TMEM_WAIT_LD(v);
+        MOE_TMEM_WAIT_LD(u);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int ew = static_cast<int>((ws4[c * 16 + j] >> (8 * g)) & 0xFFu);
-            acc[c * 16 + j] = fmaf(__uint_as_float(v[j]), exp2_int(ea + ew - 254), acc[c * 16 + j]);
+        for (int j = 0; j < 32; ++j) {
+            const int ew = static_cast<int>((ws4[c * 64 + j] >> (8 * g)) & 0xFFu);
+            acc[c * 64 + j] = fmaf(__uint_as_float(v[j]), exp2_int(ea + ew - 254), acc[c * 64 + j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int ew = static_cast<int>((ws4[c * 64 + 32 + j] >> (8 * g)) & 0xFFu);
+            acc[c * 64 + 32 + j] = fmaf(__uint_as_float(u[j]), exp2_int(ea + ew - 254), acc[c * 64 + 32 + j]);
         }
     }
 }
@@ -167,9 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int GPS = RECIPE == 0 ? 1 : 4;     // scale groups per stage
     constexpr int MPG = 4 / GPS;                 // K=32 MMAs per scale group
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
+    if (warp < kFirstEpiWarp) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+        if (warp == 0 && lane == 0) {
+            // -------------------------------------------------------------- TMA producer
             uint32_t it = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
@@ -180,27 +206,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ws_bytes = static_cast<uint32_t>(min(kTileN, p.N - nb * kTileN)) * 4u;
                 const uint8_t* ws_src = static_cast<const uint8_t*>(p.w_scale) +
                                         (static_cast<size_t>(e) * KB * p.N + static_cast<size_t>(nb) * kTileN) * 4;
+                // activation scales are stored [K/128][a_pad]: one 16-byte-aligned run per stage
+                const uint8_t* sa_src = static_cast<const uint8_t*>(p.a_scale) + static_cast<size_t>(row0 & ~3) * 4;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % kStages;
                     if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + ws_bytes);
+                    mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + ws_bytes + kSaBytes);
                     tma_load_2d(smem + L::a + s * kABytes, &tmA, kb * kTileK, row0, &full[s]);
                     tma_load_2d(smem + L::b + s * kBBytes, &tmB, kb * kTileK, brow0, &full[s]);
-                    bulk_load(smem + L::ws + s * kWsBytes, ws_src + static_cast<size_t>(kb) * p.N * 4, ws_bytes,
+                    bulk_load(smem + L::sc + s * kScaleSlot, ws_src + static_cast<size_t>(kb) * p.N * 4, ws_bytes,
                               &full[s]);
+                    bulk_load(smem + L::sc + s * kScaleSlot + kWsBytes,
+                              sa_src + static_cast<size_t>(kb) * p.a_pad * 4, kSaBytes, &full[s]);
                 }
             }
             if (!ok) {   // let the copies already issued land before the CTA leaves
                 const uint32_t n = it < static_cast<uint32_t>(kStages) ? it : kStages;
                 for (uint32_t i = it - n; i < it; ++i) drain_wait(&full[i % kStages], (i / kStages) & 1);
             }
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        } else if (warp == 1 && lane == 0) {
+            // -------------------------------------------------------------- MMA issuer
             const uint32_t idesc = f8_idesc(kTileM, kTileN);
             uint32_t it = 0, kg = 0;
             bool ok = true;
@@ -236,8 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             drain_wait(drain, 0);
         }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
         // ------------------------------------------------------------------ epilogue
-        const int ew = warp - 2;
+        const int ew = warp - kFirstEpiWarp;
         const int quad = warp & 3;                // TMEM lanes 32*quad .. 32*quad+31
         const int half = ew >> 2;                 // columns half*128 .. half*128+127 of the tile
         const int row_in_tile = quad * 32 + lane;
@@ -258,18 +287,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             for (int kb = 0; kb < KB && ok; ++kb, ++it) {
                 const int s = it % kStages;
-                float sa = 0.0f;
-                uint32_t sa4 = 0;
-                if (row_ok) {
-                    if (RECIPE == 0) sa = static_cast<const float*>(p.a_scale)[static_cast<size_t>(r) * KB + kb];
-                    else sa4 = static_cast<const uint32_t*>(p.a_scale)[static_cast<size_t>(r) * KB + kb];
-                }
-                // acquire the stage (its weight scales were written by the bulk copy)
+                // acquire the stage (its scales were written by the bulk copies)
                 if (!mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
-                const uint8_t* ws_stage = smem + L::ws + s * kWsBytes + half * 128 * 4;
+                const uint8_t* ws_stage = smem + L::sc + s * kScaleSlot + half * 128 * 4;
+                const uint32_t saw = reinterpret_cast<const uint32_t*>(smem + L::sc + s * kScaleSlot + kWsBytes)
+                    [(row0 & 3) + row_in_tile];
+                const float sa = __uint_as_float(saw);
+                const uint32_t sa4 = saw;
                 for (int g = 0; g < GPS; ++g, ++kg) {
                     const int b = kg & 1;
                     if (!mbar_wait(&tfull[b], (kg >> 1) & 1, abort_flag, p.status)) {
@@ -301,13 +328,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int I = p.N >> 1;
                 const int c0 = nb * 128 + half * 64;
                 if (warp_active) {
+                    if (p.bias) {
+                        const uint4* bg = reinterpret_cast<const uint4*>(p.bias + static_cast<size_t>(e) * p.N + c0);
+                        const uint4* bu = reinterpret_cast<const uint4*>(p.bias + static_cast<size_t>(e) * p.N + I + c0);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            const uint4 g4 = __ldg(bg + v), u4 = __ldg(bu + v);
+                            const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w}, uw[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                acc[8 * v + 2 * q] += __uint_as_float(gw[q] << 16);
+                                acc[8 * v + 2 * q + 1] += __uint_as_float(gw[q] & 0xFFFF0000u);
+                                acc[64 + 8 * v + 2 * q] += __uint_as_float(uw[q] << 16);
+                                acc[64 + 8 * v + 2 * q + 1] += __uint_as_float(uw[q] & 0xFFFF0000u);
+                            }
+                        }
+                    }
 #pragma unroll
                     for (int i = 0; i < 64; ++i) {
-                        float gt = acc[i], up = acc[64 + i];
-                        if (p.bias) {
-                            gt += __bfloat162float(p.bias[static_cast<size_t>(e) * p.N + c0 + i]);
-                            up += __bfloat162float(p.bias[static_cast<size_t>(e) * p.N + I + c0 + i]);
-                        }
+                        const float gt = acc[i], up = acc[64 + i];
                         acc[i] = __fdiv_rn(gt, 1.0f + expf(-gt)) * up;
                     }
                 }
@@ -340,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          __fdiv_rn(acc[16 * w + 14], sc), __fdiv_rn(acc[16 * w + 15], sc));
                             dst[w] = q;
                         }
-                        if (half == 0) static_cast<float*>(p.act_s)[static_cast<size_t>(r) * (I >> 7) + nb] = sc;
+                        if (half == 0) static_cast<float*>(p.act_s)[static_cast<size_t>(nb) * p.a_pad + r] = sc;
                     }
                 } else if (warp_active && row_ok) {
                     uint32_t* dst = reinterpret_cast<uint32_t*>(p.act_q + static_cast<size_t>(r) * I + c0);
@@ -359,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint4* d4 = reinterpret_cast<uint4*>(dst + 8 * grp);
                         d4[0] = make_uint4(q[0], q[1], q[2], q[3]);
                         d4[1] = make_uint4(q[4], q[5], q[6], q[7]);
-                        static_cast<uint8_t*>(p.act_s)[static_cast<size_t>(r) * (I >> 5) + nb * 4 + half * 2 + grp] =
+                        static_cast<uint8_t*>(p.act_s)[(static_cast<size_t>(nb) * p.a_pad + r) * 4 + half * 2 + grp] =
                             static_cast<uint8_t>(ex + 127);
                     }
                 }
@@ -368,18 +407,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int c0 = nb * kTileN + half * 128;
                 if (warp_active && row_ok && c0 < p.N) {
                     float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.N + c0);
+                    if (p.bias) {
+                        const uint4* bb = reinterpret_cast<const uint4*>(p.bias + static_cast<size_t>(e) * p.N + c0);
 #pragma unroll
-                    for (int c = 0; c < 128; c += 4) {
-                        float4 v = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-                        if (p.bias) {
-                            const __nv_bfloat16* bb = p.bias + static_cast<size_t>(e) * p.N + c0 + c;
-                            v.x += __bfloat162float(bb[0]);
-                            v.y += __bfloat162float(bb[1]);
-                            v.z += __bfloat162float(bb[2]);
-                            v.w += __bfloat162float(bb[3]);
+                        for (int v = 0; v < 16; ++v) {
+                            const uint4 b4 = __ldg(bb + v);
+                            const uint32_t bw[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                acc[8 * v + 2 * q] += __uint_as_float(bw[q] << 16);
+                                acc[8 * v + 2 * q + 1] += __uint_as_float(bw[q] & 0xFFFF0000u);
+                            }
                         }
-                        dst[c >> 2] = v;
                     }
+#pragma unroll
+                    for (int c = 0; c < 128; c += 4) dst[c >> 2] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
                 }
             }
         }
@@ -397,8 +439,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int MODE, int RECIPE>
 static cudaError_t launch_gemm_t(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
                                  cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm<MODE, RECIPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kSmemBytes));
+    // The register split above must fit what the block is launched with, or setmaxnreg.inc
+    // would wait forever: refuse to launch otherwise.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, k_grouped_gemm<MODE, RECIPE>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * kThreads < kRegsLow * 128 + kRegsHigh * 256) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(k_grouped_gemm<MODE, RECIPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
     k_grouped_gemm<MODE, RECIPE><<<num_sms, kThreads, kSmemBytes, s>>>(tmA, tmB, a);
     return cudaGetLastError();

@@ -39,9 +39,9 @@ struct QuantArgs {
     const __nv_bfloat16* x;     // [T, H]
     const int32_t* row_of;      // [T, K]
     uint8_t* xq;                // [A, H]
-    void* xs;                   // [A, H/g]
+    void* xs;                   // [H/128][a_pad] 4-byte words (fp32, or 4 x UE8M0)
     int32_t* status;
-    int T, H, K, recipe;
+    int T, H, K, recipe, a_pad;
 };
 
 struct CombineArgs {
@@ -62,13 +62,14 @@ struct GemmArgs {
     int mode;                   // 0: gate+up, SwiGLU, requantize; 1: down projection
     int recipe;
     int N, K, E, A;
+    int a_pad;                  // row stride of the stage-major activation scales
     const int32_t* offsets;     // [E + 1]
     const int32_t* tile_start;  // [E + 1]
-    const void* a_scale;        // [A, K/g]
+    const void* a_scale;        // [K/128][a_pad] 4-byte words: fp32, or 4 x UE8M0 (one per 32-block)
     const void* w_scale;        // recipe 0: fp32 [E, K/128, N]; recipe 1: u8 [E, K/128, N, 4]
     const __nv_bfloat16* bias;  // [E, N] in the caller's column order, or null
     uint8_t* act_q;             // mode 0: [A, N/2]
-    void* act_s;                // mode 0: [A, (N/2)/g]
+    void* act_s;                // mode 0: [(N/2)/128][a_pad] 4-byte words
     float* out;                 // mode 1: [A, N]
     int32_t* status;
 };
@@ -80,6 +81,7 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s);
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         int num_sms, cudaStream_t s);
+int set_last_error(int code, const char* msg);
 cudaError_t launch_selftest_wait(int32_t* status, uint32_t timeout_us, cudaStream_t s);
 
 // Column permutation applied to w13 by the transform: within each 256-column block nb,

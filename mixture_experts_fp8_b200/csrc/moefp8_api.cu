@@ -46,9 +46,6 @@ int ok() {
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-int scale_group(const moe_config_t* c) { return c->recipe == 0 ? 128 : 32; }
-size_t scale_elem_bytes(const moe_config_t* c) { return c->recipe == 0 ? 4 : 1; }
-
 int check_config(const moe_config_t* c) {
     if (!c) return fail(MOE_ERR_INVALID_ARG, "config is NULL");
     if (c->num_tokens <= 0) return fail(MOE_ERR_INVALID_ARG, "num_tokens must be > 0 (got %d)", c->num_tokens);
@@ -85,9 +82,13 @@ int check_config(const moe_config_t* c) {
     return MOE_OK;
 }
 
+// Row stride of the stage-major scale arrays: every routed row, plus room for a 128-row tile
+// read starting at a 16-byte-aligned row just before the last row.
+size_t scale_rows_of(size_t A) { return align_up(A + moe::kTileM + 4, 4); }
+
 void layout_of(const moe_config_t* c, moe_workspace_layout_t* L) {
     const size_t T = c->num_tokens, K = c->top_k, E = c->num_experts, H = c->hidden, I = c->inter;
-    const size_t A = T * K, g = scale_group(c), sb = scale_elem_bytes(c);
+    const size_t A = T * K, SR = scale_rows_of(A);
     const size_t chunks = (A + moe::kPermuteChunk - 1) / moe::kPermuteChunk;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -105,10 +106,11 @@ void layout_of(const moe_config_t* c, moe_workspace_layout_t* L) {
     L->row_of = take(4 * A);
     L->hist = take(4 * chunks * E);
     L->xq = take(A * H);
-    L->xs = take(A * (H / g) * sb);
+    L->xs = take((H / 128) * SR * 4);
     L->act_q = take(A * I);
-    L->act_s = take(A * (I / g) * sb);
+    L->act_s = take((I / 128) * SR * 4);
     L->o = take(4 * A * H);
+    L->scale_rows = SR;
     L->total = off;
 }
 
@@ -172,6 +174,14 @@ int make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t co
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 }  // namespace
+
+namespace moe {
+// Record a message as the calling thread's last error (for entry points in other files).
+int set_last_error(int code, const char* msg) {
+    g_err = msg ? msg : "";
+    return code;
+}
+}  // namespace moe
 
 // ============================================================================ profiler
 struct moe_profile {
@@ -285,10 +295,10 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     if (!aligned(hidden_states, 16) || !aligned(y, 16) || !aligned(w13_t, 16) || !aligned(w2_t, 16) ||
         !aligned(w13s_t, 16) || !aligned(w2s_t, 16) || !aligned(workspace, 256) ||
         (router_logits && !aligned(router_logits, 4)) || (topk_idx && !aligned(topk_idx, 4)) ||
-        (topk_weights && !aligned(topk_weights, 4)) || (w13_bias && !aligned(w13_bias, 2)) ||
-        (w2_bias && !aligned(w2_bias, 2)) || (expert_counts && !aligned(expert_counts, 4)))
+        (topk_weights && !aligned(topk_weights, 4)) || (w13_bias && !aligned(w13_bias, 16)) ||
+        (w2_bias && !aligned(w2_bias, 16)) || (expert_counts && !aligned(expert_counts, 4)))
         return fail(MOE_ERR_INVALID_ARG,
-                    "moe_forward: misaligned buffer (hidden_states, y and weights need 16 bytes, workspace 256)");
+                    "moe_forward: misaligned buffer (hidden_states, y, weights and biases need 16 bytes, workspace 256)");
     moe_workspace_layout_t L;
     layout_of(cfg, &L);
     if (workspace_bytes < L.total)
@@ -331,7 +341,8 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     MOE_CUDA_TRY(moe::launch_permute(pa, s));
     MOE_CUDA_TRY(mark(2));
     moe::QuantArgs qa{static_cast<const __nv_bfloat16*>(hidden_states), static_cast<const int32_t*>(at(L.row_of)),
-                      static_cast<uint8_t*>(at(L.xq)), at(L.xs), status, T, H, K, cfg->recipe};
+                      static_cast<uint8_t*>(at(L.xq)), at(L.xs), status, T, H, K, cfg->recipe,
+                      static_cast<int>(L.scale_rows)};
     MOE_CUDA_TRY(moe::launch_quant(qa, s));
     MOE_CUDA_TRY(mark(3));
     moe::GemmArgs g1{};
@@ -341,6 +352,7 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     g1.K = H;
     g1.E = E;
     g1.A = A;
+    g1.a_pad = static_cast<int>(L.scale_rows);
     g1.offsets = static_cast<const int32_t*>(at(L.offsets));
     g1.tile_start = static_cast<const int32_t*>(at(L.tile_start));
     g1.a_scale = at(L.xs);

@@ -52,9 +52,9 @@ __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
         }
         *reinterpret_cast<uint32_t*>(a.xq + static_cast<size_t>(r) * a.H + cb * 128 + 4 * lane) = q;
         if (a.recipe == 0) {
-            if (lane == 0) static_cast<float*>(a.xs)[static_cast<size_t>(r) * nblk + cb] = s32;
+            if (lane == 0) static_cast<float*>(a.xs)[static_cast<size_t>(cb) * a.a_pad + r] = s32;
         } else if ((lane & 7) == 0) {
-            static_cast<uint8_t*>(a.xs)[static_cast<size_t>(r) * (a.H >> 5) + cb * 4 + (lane >> 3)] = e8;
+            static_cast<uint8_t*>(a.xs)[(static_cast<size_t>(cb) * a.a_pad + r) * 4 + (lane >> 3)] = e8;
         }
     }
 }

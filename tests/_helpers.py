@@ -89,6 +89,18 @@ class GpuProblem:
         nbytes = count * torch.tensor([], dtype=dtype).element_size()
         return self.workspace[off:off + nbytes].view(dtype)
 
+    def ws_scales(self, name, kdim):
+        """Scales of workspace region `name` (stored [kdim/128][scale_rows] 4-byte words) as
+        [A, kdim/g]: fp32 for recipe 0, UE8M0 bytes for recipe 1."""
+        SR = self.layout["scale_rows"]
+        nb = kdim // 128
+        A = self.shape.num_tokens * self.shape.top_k
+        words = self.ws_region(name, torch.int32, nb * SR).cpu().numpy().reshape(nb, SR)[:, :A]
+        if self.shape.recipe == 0:
+            return np.ascontiguousarray(words.view(np.float32).T)
+        b = np.ascontiguousarray(words).view(np.uint8).reshape(nb, A, 4)
+        return np.ascontiguousarray(b.transpose(1, 0, 2).reshape(A, nb * 4))
+
     def status(self) -> int:
         return self.moe.read_status(self.workspace)
 

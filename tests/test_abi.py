@@ -68,7 +68,8 @@ def test_valid_configs_and_sizes():
         assert lay["total"] == moe.workspace_size(c)
         A = s.num_tokens * s.top_k
         assert lay["o"] + 4 * A * s.hidden <= lay["total"]
-        assert all(v % 1024 == 0 for k, v in lay.items() if k != "total")
+        assert all(v % 1024 == 0 for k, v in lay.items() if k not in ("total", "scale_rows"))
+        assert lay["scale_rows"] >= A and lay["scale_rows"] % 4 == 0
         w13, w13s, w2, w2s = moe.transformed_weights_size(c)
         assert w13 == s.num_experts * s.hidden * 2 * s.inter and w2 == s.num_experts * s.inter * s.hidden
         assert w13s == s.num_experts * (s.hidden // 128) * 2 * s.inter * 4

@@ -81,10 +81,8 @@ def test_permutation_and_quantization(problems, name):
     assert np.array_equal(np.diff(tiles), (counts + 127) // 128)
 
     # quantized activations, in permuted order
-    g = shape.group
-    sdt = torch.float32 if shape.recipe == 0 else torch.uint8
     xq = gp.ws_region("xq", torch.uint8, A * H).cpu().numpy().reshape(A, H)
-    xs = gp.ws_region("xs", sdt, A * (H // g)).cpu().numpy().reshape(A, H // g)
+    xs = gp.ws_scales("xs", H)
     tok = _sample(T, 512, 5)
     tok = np.arange(T) if tok is None else tok
     q_ref, s_ref = oracle.quantize_tokens(ni["x"][tok], shape.recipe)
@@ -103,13 +101,11 @@ def test_gate_up_swiglu_codes(problems, name):
     shape = gp.shape
     T, K, I = shape.num_tokens, shape.top_k, shape.inter
     A = T * K
-    g = shape.group
     idx, w, _ = oracle.route(oracle_cfg(shape), ni["logits"], ni["per_expert_scale"])
     gp.forward(topk_idx=torch.from_numpy(idx).cuda(), topk_weights=torch.from_numpy(w).cuda())
     _, _, _, row_of = oracle.permute(idx, shape.num_experts)
-    sdt = torch.float32 if shape.recipe == 0 else torch.uint8
     aq = gp.ws_region("act_q", torch.uint8, A * I).cpu().numpy().reshape(A, I)
-    as_ = gp.ws_region("act_s", sdt, A * (I // g)).cpu().numpy().reshape(A, I // g)
+    as_ = gp.ws_scales("act_s", I)
     tok = _sample(T, 32, 3)
     tok = np.arange(min(T, 32)) if tok is None else tok
     _, rq, rs = oracle.forward(oracle_cfg(shape), ni["x"], ni["w13"], ni["w13s"], ni["w2"], ni["w2s"],
