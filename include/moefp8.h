@@ -171,6 +171,31 @@ int moe_forward(const moe_config_t *cfg, const void *hidden_states, const float 
                 const void *w13_bias, const void *w2_bias, void *y, int32_t *expert_counts,
                 void *workspace, size_t workspace_bytes, void *stream);
 
+/* moe_forward without a caller workspace, for callers that cannot allocate device memory: code
+ * running inside a host framework that owns all device memory (a serving engine's pre-reserved
+ * pool, a plugin interface that gives its kernels no scratch), where cudaMalloc is not allowed
+ * because it can synchronize the device and can fail under memory pressure mid-serving.
+ * The pages have no counterpart of this entry point.
+ *   Arguments as moe_forward, minus workspace / workspace_bytes.  The caller still owns and
+ *   passes every input and output; the scratch is a fixed 16 MiB array in the library's device
+ *   image (each GPU that loads the library holds it until the process exits).  A problem whose
+ *   moe_workspace_size exceeds 16 MiB (16777216 bytes) is rejected with MOE_ERR_UNSUPPORTED
+ *   and nothing is launched; e.g. the 64-token decode problem (H 2816, I 768, E 128, top-8)
+ *   needs about 7.7 MB.
+ *   The first call on a device looks the array's address up (cudaGetSymbolAddress) with that
+ *   device current; make that first call before any stream capture.  The array is shared by
+ *   every call on the device and keeps the last call's contents (the forward clears its status
+ *   word itself); calls that overlap on the GPU race on it.  Allocates nothing: no cudaMalloc,
+ *   no cudaFree, no allocating library routine.  The status word (moe_read_status) lives in
+ *   the array, so it cannot be read through this entry point's API; errors are still reported
+ *   by the return code. */
+int moe_forward_static_workspace(const moe_config_t *cfg, const void *hidden_states,
+                                 const float *router_logits, const float *per_expert_scale,
+                                 const int32_t *topk_idx, const float *topk_weights,
+                                 const void *w13_t, const void *w13s_t, const void *w2_t,
+                                 const void *w2s_t, const void *w13_bias, const void *w2_bias,
+                                 void *y, int32_t *expert_counts, void *stream);
+
 /* moe_forward, recording a CUDA event before each of the MOE_NUM_STAGES stages and after the
  * last one into `prof` (which accumulates per-stage device time until reset).  prof may be
  * NULL, which makes this identical to moe_forward. */

@@ -7,7 +7,8 @@ built in-tree with nvcc, and if that is impossible, importing this package fails
 
 Entry points (same names as the C ABI):
     check_config, transformed_weights_size, transform_weights, workspace_size,
-    workspace_layout, route, forward, forward_profiled, read_status, selftest_bounded_wait,
+    workspace_layout, route, forward, forward_profiled, forward_static_workspace, read_status,
+    selftest_bounded_wait,
     Profile (moe_profile_create / read / reset / destroy).
 """
 from __future__ import annotations
@@ -33,7 +34,7 @@ EXPORTED = (
     "moe_last_error", "moe_check_config", "moe_transformed_weights_size", "moe_transform_weights",
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_forward", "moe_forward_profiled",
     "moe_profile_create", "moe_profile_destroy", "moe_profile_read", "moe_profile_reset",
-    "moe_read_status", "moe_selftest_bounded_wait",
+    "moe_read_status", "moe_selftest_bounded_wait", "moe_forward_static_workspace",
 )
 
 
@@ -123,6 +124,7 @@ def _load():
             "moe_profile_reset": [P],
             "moe_read_status": [P, P, P],
             "moe_selftest_bounded_wait": [P, ctypes.c_uint32, P],
+            "moe_forward_static_workspace": [CP] + [P] * 13 + [P],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -231,6 +233,23 @@ def forward(cfg: Config, hidden_states, weights, router_logits=None, per_expert_
         _check(_load().moe_forward(*args, _stream(stream)))
     else:
         _check(_load().moe_forward_profiled(*args, profile.handle, _stream(stream)))
+    return y
+
+
+def forward_static_workspace(cfg: Config, hidden_states, weights, router_logits=None,
+                             per_expert_scale=None, topk_idx=None, topk_weights=None, w13_bias=None,
+                             w2_bias=None, y=None, expert_counts=None, stream=None):
+    """The layer forward with its scratch in the library's fixed device array (no workspace
+    argument, nothing allocated by the library).  For callers that may not allocate device
+    memory; `y` should be preallocated by such callers."""
+    import torch
+    if y is None:
+        y = torch.empty((cfg.num_tokens, cfg.hidden), dtype=torch.bfloat16, device=hidden_states.device)
+    c = cfg.c()
+    _check(_load().moe_forward_static_workspace(
+        ctypes.byref(c), _ptr(hidden_states), _ptr(router_logits), _ptr(per_expert_scale),
+        _ptr(topk_idx), _ptr(topk_weights), *[_ptr(w) for w in weights], _ptr(w13_bias),
+        _ptr(w2_bias), _ptr(y), _ptr(expert_counts), _stream(stream)))
     return y
 
 
