@@ -213,6 +213,8 @@ def main():
     ap.add_argument("--config", default="decode", choices=sorted(synth.SHAPES))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the problem's token count (reduced cases for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -220,6 +222,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     shape = synth.SHAPES[args.config]
+    if args.tokens:
+        shape = shape.with_tokens(args.tokens)
 
     if args.impl == "reference":
         reference_arm(args, shape, rank)

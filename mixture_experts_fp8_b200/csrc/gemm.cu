@@ -15,8 +15,8 @@
 //   warp 1   MMA issuer (one thread): tcgen05.mma.kind::f8f6f4, M=128 N=256 K=32.  Each scale
 //            group (128 deep for recipe 0, 32 for recipe 1) is accumulated alone into one of two
 //            256-column fp32 TMEM buffers.
-//   warps 2-3 idle.  Warpgroup 0 gives registers back (setmaxnreg.dec to 40).
-//   warps 4-11 epilogue (setmaxnreg.inc to 232): a warp reads its 32 TMEM lanes (= tile rows),
+//   warps 2-3 idle.  Warpgroup 0 gives registers back (setmaxnreg.dec to 56).
+//   warps 4-11 epilogue (setmaxnreg.inc to 224): a warp reads its 32 TMEM lanes (= tile rows),
 //            half of the columns each;
 //            every group partial is multiplied by a_s * w_s and added into fp32 registers (the
 //            "promotion"), then the tile's epilogue runs from registers.
@@ -36,7 +36,7 @@ constexpr int kStages = 4;
 constexpr int kThreads = 384;
 constexpr int kEpiWarps = 8;
 constexpr int kFirstEpiWarp = 4;
-constexpr int kRegsLow = 40, kRegsHigh = 232;      // 128 * 40 + 256 * 232 = 384 * 168 (65536 / 384 -> 168)
+constexpr int kRegsLow = 56, kRegsHigh = 224;      // 128 * 56 + 256 * 224 = 384 * 168 (65536 / 384 -> 168)
 constexpr uint32_t kABytes = kTileM * kTileK;      // 16 KB
 constexpr uint32_t kBBytes = kTileN * kTileK;      // 32 KB
 constexpr uint32_t kWsBytes = kTileN * 4;          // weight scales: fp32 or 4 x UE8M0 per column
@@ -85,38 +85,45 @@ __device__ __forceinline__ void decode_unit(int u, int nt, const int* tstart, in
     mb = local - nb * mt;
 }
 
-// acc[j] += P[j] * (sa * ws[j]) for the 128 columns of this thread's half: two rounds of two
-// 32-column TMEM loads, one wait each.
-__device__ __forceinline__ void promote_fp32(float (&acc)[128], uint32_t taddr, const float* ws, float sa) {
+// acc[j] += P[j] * (sa * ws[j]) over 32 columns [c0, c0 + 32) already loaded into v; packed
+// fp32x2 multiply and FMA (each lane rounds as the scalar operations would).
+__device__ __forceinline__ void fma_chunk32(float2 (&acc)[64], const uint32_t (&v)[32], const float* ws, int c0,
+                                            float2 sa2) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-        uint32_t v[32], u[32];
-        MOE_TMEM_LD32(taddr + c * 64, v);
-        MOE_TMEM_LD32(taddr + c * 64 + 32, u);
-        MOE_TMEM_WAIT_LD(v);
-        MOE_TMEM_WAIT_LD(u);
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            const float4 w4 = *reinterpret_cast<const float4*>(ws + c * 64 + j);
-            acc[c * 64 + j + 0] = fmaf(__uint_as_float(v[j + 0]), sa * w4.x, acc[c * 64 + j + 0]);
-            acc[c * 64 + j + 1] = fmaf(__uint_as_float(v[j + 1]), sa * w4.y, acc[c * 64 + j + 1]);
-            acc[c * 64 + j + 2] = fmaf(__uint_as_float(v[j + 2]), sa * w4.z, acc[c * 64 + j + 2]);
-            acc[c * 64 + j + 3] = fmaf(__uint_as_float(v[j + 3]), sa * w4.w, acc[c * 64 + j + 3]);
-        }
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-            const float4 w4 = *reinterpret_cast<const float4*>(ws + c * 64 + 32 + j);
-            acc[c * 64 + 32 + j + 0] = fmaf(__uint_as_float(u[j + 0]), sa * w4.x, acc[c * 64 + 32 + j + 0]);
-            acc[c * 64 + 32 + j + 1] = fmaf(__uint_as_float(u[j + 1]), sa * w4.y, acc[c * 64 + 32 + j + 1]);
-            acc[c * 64 + 32 + j + 2] = fmaf(__uint_as_float(u[j + 2]), sa * w4.z, acc[c * 64 + 32 + j + 2]);
-            acc[c * 64 + 32 + j + 3] = fmaf(__uint_as_float(u[j + 3]), sa * w4.w, acc[c * 64 + 32 + j + 3]);
-        }
+    for (int j = 0; j < 32; j += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(ws + c0 + j);
+        const float2 s0 = __fmul2_rn(make_float2(w4.x, w4.y), sa2);
+        const float2 s1 = __fmul2_rn(make_float2(w4.z, w4.w), sa2);
+        acc[(c0 + j) / 2] = __ffma2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), s0,
+                                       acc[(c0 + j) / 2]);
+        acc[(c0 + j) / 2 + 1] = __ffma2_rn(make_float2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])), s1,
+                                           acc[(c0 + j) / 2 + 1]);
     }
 }
 
+// The promotion of one scale group over this thread's 128 columns: four 32-column TMEM loads,
+// two in flight while the previous two are multiplied in.
+__device__ __forceinline__ void promote_fp32(float2 (&acc)[64], uint32_t taddr, const float* ws, float sa) {
+    const float2 sa2 = make_float2(sa, sa);
+    uint32_t v[32], u[32];
+    MOE_TMEM_LD32(taddr, v);
+    MOE_TMEM_LD32(taddr + 32, u);
+    MOE_TMEM_WAIT_LD(v);
+    MOE_TMEM_WAIT_LD(u);
+    fma_chunk32(acc, v, ws, 0, sa2);
+    MOE_TMEM_LD32(taddr + 64, v);
+    fma_chunk32(acc, u, ws, 32, sa2);
+    MOE_TMEM_LD32(taddr + 96, u);
+    MOE_TMEM_WAIT_LD(v);
+    MOE_TMEM_WAIT_LD(u);
+    fma_chunk32(acc, v, ws, 64, sa2);
+    fma_chunk32(acc, u, ws, 96, sa2);
+}
+
 // Same with UE8M0 scales: the scale is 2^(ea + ew - 254), exact.
-__device__ __forceinline__ void promote_mx(float (&acc)[128], uint32_t taddr, const uint32_t* ws4, int ea,
+__device__ __forceinline__ void promote_mx(float2 (&acc2)[64], uint32_t taddr, const uint32_t* ws4, int ea,
                                            int g) {
+    float* acc = reinterpret_cast<float*>(acc2);
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
         uint32_t v[32], u[32];
@@ -145,8 +152,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const GemmArgs p) {
     extern __shared__ uint8_t smem_raw[];
     const int nt = (p.N + kTileN - 1) / kTileN;
-    const int total_units = p.tile_start[p.E] * nt;
-    if (static_cast<int>(blockIdx.x) >= total_units) return;
 
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -163,10 +168,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* s_off = reinterpret_cast<int*>(smem + L::off);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i <= p.E; i += kThreads) {
-        s_tstart[i] = p.tile_start[i];
-        s_off[i] = p.offsets[i];
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
@@ -184,10 +185,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmB);
     }
     if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
+    // everything above overlaps the previous kernel; its outputs are read only from here on
+    pdl_wait_then_release();
+    for (int i = threadIdx.x; i <= p.E; i += kThreads) {
+        s_tstart[i] = p.tile_start[i];
+        s_off[i] = p.offsets[i];
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    const int total_units = s_tstart[p.E] * nt;
     const int KB = p.K / kTileK;                 // pipeline stages per unit
     constexpr int GPS = RECIPE == 0 ? 1 : 4;     // scale groups per stage
     constexpr int MPG = 4 / GPS;                 // K=32 MMAs per scale group
@@ -281,9 +289,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_ok = row_in_tile < cnt;
             const int r = row0 + row_in_tile;
 
-            float acc[128];
+            float2 acc2[64];
 #pragma unroll
-            for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+            for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
+            float* acc = reinterpret_cast<float*>(acc2);
 
             for (int kb = 0; kb < KB && ok; ++kb, ++it) {
                 const int s = it % kStages;
@@ -308,9 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                                static_cast<uint32_t>(b * kTileN + half * 128);
                         if (RECIPE == 0)
-                            promote_fp32(acc, taddr, reinterpret_cast<const float*>(ws_stage), sa);
+                            promote_fp32(acc2, taddr, reinterpret_cast<const float*>(ws_stage), sa);
                         else
-                            promote_mx(acc, taddr, reinterpret_cast<const uint32_t*>(ws_stage),
+                            promote_mx(acc2, taddr, reinterpret_cast<const uint32_t*>(ws_stage),
                                        static_cast<int>((sa4 >> (8 * g)) & 0xFFu), g);
                     }
                     tc_fence_before();
@@ -448,8 +457,7 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, const CUtensorMap& tmA, cons
     e = cudaFuncSetAttribute(k_grouped_gemm<MODE, RECIPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
-    k_grouped_gemm<MODE, RECIPE><<<num_sms, kThreads, kSmemBytes, s>>>(tmA, tmB, a);
-    return cudaGetLastError();
+    return launch_pdl(k_grouped_gemm<MODE, RECIPE>, dim3(num_sms), dim3(kThreads), kSmemBytes, s, tmA, tmB, a);
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,

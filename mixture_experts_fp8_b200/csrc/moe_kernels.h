@@ -8,7 +8,7 @@
 
 namespace moe {
 
-constexpr int kPermuteChunk = 1024;   // routed rows per histogram / scatter chunk
+constexpr int kPermuteChunk = 256;    // routed rows per histogram / scatter chunk
 constexpr int kTileM = 128;           // GEMM rows per tile
 constexpr int kTileN = 256;           // GEMM output columns per tile
 constexpr int kTileK = 128;           // K bytes (= E4M3 elements) per pipeline stage

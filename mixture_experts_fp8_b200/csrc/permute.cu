@@ -16,6 +16,7 @@ namespace moe {
 
 __global__ void __launch_bounds__(256) k_hist(PermuteArgs a) {
     __shared__ int cnt[MOE_MAX_EXPERTS];
+    pdl_wait_then_release();
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
     const int begin = blockIdx.x * kPermuteChunk;
@@ -59,6 +60,7 @@ __device__ int block_exclusive_scan_256(int v, int* tmp) {
 
 __global__ void __launch_bounds__(256) k_scan(PermuteArgs a) {
     __shared__ int tmp[16];
+    pdl_wait_then_release();
     const int e = threadIdx.x;
     int run = 0;
     if (e < a.E) {
@@ -87,16 +89,25 @@ __global__ void __launch_bounds__(256) k_scan(PermuteArgs a) {
 
 __global__ void __launch_bounds__(32) k_scatter(PermuteArgs a) {
     __shared__ int base[MOE_MAX_EXPERTS];
+    constexpr int kBatches = kPermuteChunk / 32;
+    pdl_wait_then_release();
     const int lane = threadIdx.x;
+    const int begin = blockIdx.x * kPermuteChunk;
+    const int end = min(a.A, begin + kPermuteChunk);
+    int ids[kBatches];                                  // all of the chunk's ids, loaded at once
+#pragma unroll
+    for (int b = 0; b < kBatches; ++b) {
+        const int r = begin + 32 * b + lane;
+        ids[b] = r < end ? a.idx[r] : -1;
+    }
     for (int e = lane; e < a.E; e += 32)
         base[e] = a.offsets[e] + a.hist[static_cast<size_t>(blockIdx.x) * a.E + e];
     __syncwarp();
-    const int begin = blockIdx.x * kPermuteChunk;
-    const int end = min(a.A, begin + kPermuteChunk);
-    for (int r0 = begin; r0 < end; r0 += 32) {
-        const int r = r0 + lane;
+#pragma unroll
+    for (int b = 0; b < kBatches; ++b) {
+        const int r = begin + 32 * b + lane;
         const bool valid = r < end;
-        int e = valid ? a.idx[r] : -1;
+        int e = ids[b];
         if (e >= a.E) e = -1;                           // reported by k_hist
         const uint32_t active = __ballot_sync(0xffffffffu, valid && e >= 0);
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
@@ -115,10 +126,10 @@ __global__ void __launch_bounds__(32) k_scatter(PermuteArgs a) {
 }
 
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
-    k_hist<<<a.chunks, 256, 0, s>>>(a);
-    k_scan<<<1, 256, 0, s>>>(a);
-    k_scatter<<<a.chunks, 32, 0, s>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(k_hist, dim3(a.chunks), dim3(256), 0, s, a);
+    if (e == cudaSuccess) e = launch_pdl(k_scan, dim3(1), dim3(256), 0, s, a);
+    if (e == cudaSuccess) e = launch_pdl(k_scatter, dim3(a.chunks), dim3(32), 0, s, a);
+    return e;
 }
 
 }  // namespace moe

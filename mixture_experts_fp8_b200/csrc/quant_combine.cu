@@ -18,6 +18,7 @@ namespace moe {
 
 // One warp per (token, 128-column block).  Lane l owns columns 4l .. 4l+3 of the block.
 __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
+    pdl_wait_then_release();
     const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     const int nblk = a.H >> 7;
@@ -61,14 +62,15 @@ __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s) {
     const int warps = a.T * (a.H >> 7);
-    k_quant<<<(warps + 7) / 8, 256, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k_quant, dim3((warps + 7) / 8), dim3(256), 0, s, a);
 }
 
-// One block per token; thread i handles float4 columns i, i + 256, ...
+// Grid (token, column block): thread i of block (t, cb) handles float4 column cb * 256 + i, so
+// every routed row's loads are in flight at once.
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
     __shared__ int s_row[MOE_MAX_EXPERTS];
     __shared__ float s_w[MOE_MAX_EXPERTS];
+    pdl_wait_then_release();
     const int t = blockIdx.x;
     const int A = a.T * a.K;
     for (int j = threadIdx.x; j < a.K; j += blockDim.x) {
@@ -77,29 +79,28 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
         s_w[j] = a.w[static_cast<size_t>(t) * a.K + j];
     }
     __syncthreads();
-    const int H4 = a.H >> 2;
-    for (int c = threadIdx.x; c < H4; c += blockDim.x) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < a.K; ++j) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(a.o + static_cast<size_t>(s_row[j]) * a.H) + c);
-            const float w = s_w[j];
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
-        }
-        __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-        __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-        uint2 out;
-        out.x = *reinterpret_cast<uint32_t*>(&lo);
-        out.y = *reinterpret_cast<uint32_t*>(&hi);
-        reinterpret_cast<uint2*>(a.y + static_cast<size_t>(t) * a.H)[c] = out;
+    const int c = blockIdx.y * blockDim.x + threadIdx.x;
+    if (c >= (a.H >> 2)) return;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < a.K; ++j) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(a.o + static_cast<size_t>(s_row[j]) * a.H) + c);
+        const float w = s_w[j];
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
     }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 out;
+    out.x = *reinterpret_cast<uint32_t*>(&lo);
+    out.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(a.y + static_cast<size_t>(t) * a.H)[c] = out;
 }
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
-    k_combine<<<a.T, 256, 0, s>>>(a);
-    return cudaGetLastError();
+    const int cblocks = ((a.H >> 2) + 255) / 256;
+    return launch_pdl(k_combine, dim3(a.T, cblocks), dim3(256), 0, s, a);
 }
 
 // ------------------------------------------------------------------------------------------

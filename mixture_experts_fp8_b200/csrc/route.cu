@@ -38,6 +38,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route(RouteArgs a) {
     __shared__ int s_sel[kRouteWarps][256];
     __shared__ unsigned char s_elig[kRouteWarps][256];
 
+    pdl_wait_then_release();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * kRouteWarps + warp;
     if (t >= a.T) return;
@@ -132,7 +133,10 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route(RouteArgs a) {
         }
         argmax_reduce(bv, bi);
         if (bi >= 0 && (bi & 31) == lane) avail &= ~(1u << (bi >> 5));
-        if (lane == 0) s_sel[warp][j] = bi;
+        if (lane == 0) {
+            s_sel[warp][j] = bi;
+            s_score[warp][j] = bv;                       // the selected logit
+        }
     }
     __syncwarp();
 
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route(RouteArgs a) {
         float* wv = s_gscore[warp];
         float sum = 0.0f;
         for (int j = 0; j < K; ++j) {
-            const float lj = l[s_sel[warp][j]];
+            const float lj = s_score[warp][j];
             const float v = a.routing == 1 ? 1.0f / (1.0f + expf(-lj)) : expf(lj - m) / z;
             wv[j] = v;
             sum += v;
@@ -161,8 +165,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route(RouteArgs a) {
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
     const int blocks = (a.T + kRouteWarps - 1) / kRouteWarps;
-    k_route<<<blocks, kRouteWarps * 32, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k_route, dim3(blocks), dim3(kRouteWarps * 32), 0, s, a);
 }
 
 }  // namespace moe
