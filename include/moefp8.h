@@ -124,7 +124,7 @@ int moe_transformed_weights_size(const moe_config_t *cfg, size_t *w13_bytes, siz
  *   w2_scale   device, recipe 0: fp32 [E, I/128, H];  recipe 1: UE8M0 bytes [E, I/32, H]
  * (scales are K-block-major, the orientation of the "MindIE-SD Fused MoE" MXFP8 example.)
  * Outputs (device, sizes from moe_transformed_weights_size; opaque to the caller): K-major
- * codes with gate/up columns interleaved in 64-column blocks, and the scales re-laid to match.
+ * codes with gate/up columns interleaved in 32-column blocks, and the scales re-laid to match.
  * Inputs and outputs must not overlap. */
 int moe_transform_weights(const moe_config_t *cfg, const void *w13, const void *w13_scale,
                           const void *w2, const void *w2_scale, void *w13_t, void *w13s_t,

@@ -9,34 +9,39 @@
 // quantized SiLU products, then the down projection; "MATE Mega MoE", API: swiglu;
 // "MindIE-SD Fused MoE", parameter table: w13_bias / w2_bias.
 //
-// Design (one persistent CTA per SM, 384 threads = three warpgroups):
+// Design (one persistent CTA per SM, 640 threads = five warpgroups):
 //   warp 0   TMA producer: per 128-deep K stage, a 128x128 A tile and a 256x128 B tile (both
-//            K-major, 128-byte swizzle) plus the 256 weight scales of the stage (bulk copy).
+//            K-major, 128-byte swizzle), the 256 weight scales of the stage and the tile rows'
+//            activation scales (bulk copies).
 //   warp 1   MMA issuer (one thread): tcgen05.mma.kind::f8f6f4, M=128 N=256 K=32.  Each scale
 //            group (128 deep for recipe 0, 32 for recipe 1) is accumulated alone into one of two
 //            256-column fp32 TMEM buffers.
-//   warps 2-3 idle.  Warpgroup 0 gives registers back (setmaxnreg.dec to 56).
-//   warps 4-11 epilogue (setmaxnreg.inc to 224): a warp reads its 32 TMEM lanes (= tile rows),
-//            half of the columns each;
-//            every group partial is multiplied by a_s * w_s and added into fp32 registers (the
-//            "promotion"), then the tile's epilogue runs from registers.
+//   warps 2-3 idle.  Warpgroup 0 gives registers back (setmaxnreg.dec to 32).
+//   warps 4-19 epilogue (setmaxnreg.inc to 112): warp w reads TMEM lanes 32*(w%4) .. +31 (tile
+//            rows) and one quarter of the columns; every group partial is multiplied by
+//            a_s * w_s and added into fp32 registers (the "promotion"), then the tile's epilogue
+//            runs from registers.  Four warps per lane quadrant keep the TMEM reads, which are
+//            the critical path of the promotion, in parallel.
 // Work unit = (expert, 256-column block, 128-row block), enumerated expert by expert, column
 // block, then row block; CTA c takes units c, c + grid, ...  Rows past an expert's end are
 // computed on whatever the tile holds and never stored.  Every wait is bounded.
 #include <math.h>
 
-#include "moe_common.cuh"
-#include "moe_kernels.h"
+#include "gemm_common.cuh"
 
 namespace moe {
 
 namespace {
 
 constexpr int kStages = 4;
-constexpr int kThreads = 384;
-constexpr int kEpiWarps = 8;
+constexpr int kThreads = 640;
 constexpr int kFirstEpiWarp = 4;
-constexpr int kRegsLow = 56, kRegsHigh = 224;      // 128 * 56 + 256 * 224 = 384 * 168 (65536 / 384 -> 168)
+constexpr int kEpiWarps = 16;
+constexpr int kCols = kTileN / 4;                  // columns per epilogue thread
+// Registers: 640 threads launch with 96 each (5 warps per SM sub-partition); warpgroup 0 keeps
+// 32, the four epilogue warpgroups take 112: 128 * 32 + 512 * 112 = 640 * 96.
+constexpr int kRegsLaunch = 96, kRegsLow = 32, kRegsHigh = 112;
+static_assert(128 * kRegsLow + 512 * kRegsHigh == kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kABytes = kTileM * kTileK;      // 16 KB
 constexpr uint32_t kBBytes = kTileN * kTileK;      // 32 KB
 constexpr uint32_t kWsBytes = kTileN * 4;          // weight scales: fp32 or 4 x UE8M0 per column
@@ -44,7 +49,6 @@ constexpr uint32_t kSaWords = kTileM + 4;          // activation scales of the t
 constexpr uint32_t kSaBytes = kSaWords * 4;
 constexpr uint32_t kScaleSlot = 2048;              // per stage: [weight scales | activation scales]
 constexpr uint32_t kTmemCols = 2 * kTileN;         // two fp32 accumulators
-constexpr unsigned long long kDrainLimitNs = 100000000ull;
 
 struct L {
     static constexpr uint32_t a = 0;
@@ -53,20 +57,13 @@ struct L {
     static constexpr uint32_t bars = sc + kStages * kScaleSlot;
     static constexpr uint32_t nbars = 2 * kStages + 7;   // full, empty, tfull[2], tempty[2], drain, amax[2]
     static constexpr uint32_t misc = bars + nbars * 8;   // tmem holder, abort flag
-    static constexpr uint32_t amax = misc + 16;          // float [2 buffers][2 halves][128 rows]
-    static constexpr uint32_t tstart = amax + 2 * 2 * 128 * 4;
+    static constexpr uint32_t amax = misc + 16;          // float [2 buffers][4 quarters][128 rows]
+    static constexpr uint32_t tstart = amax + 2 * 4 * 128 * 4;
     static constexpr uint32_t off = tstart + (MOE_MAX_EXPERTS + 1) * 4;
     static constexpr uint32_t end = off + (MOE_MAX_EXPERTS + 1) * 4;
 };
 constexpr uint32_t kSmemBytes = L::end + 1024;   // + slack to align the base to 1024 bytes
-
-// Bounded wait used only while leaving after an abort: ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const uint32_t a = smem_u32(bar);
-    const unsigned long long t0 = globaltimer_ns();
-    while (!mbar_try_wait(a, parity))
-        if (globaltimer_ns() - t0 > kDrainLimitNs) break;
-}
+static_assert(kSmemBytes <= 232448, "shared memory");
 
 // Unit u -> (expert e, column block nb, row block mb).  Expert e owns units
 // [nt * tstart[e], nt * tstart[e+1]); empty experts own none.
@@ -87,8 +84,8 @@ __device__ __forceinline__ void decode_unit(int u, int nt, const int* tstart, in
 
 // acc[j] += P[j] * (sa * ws[j]) over 32 columns [c0, c0 + 32) already loaded into v; packed
 // fp32x2 multiply and FMA (each lane rounds as the scalar operations would).
-__device__ __forceinline__ void fma_chunk32(float2 (&acc)[64], const uint32_t (&v)[32], const float* ws, int c0,
-                                            float2 sa2) {
+__device__ __forceinline__ void fma_chunk32(float2 (&acc)[kCols / 2], const uint32_t (&v)[32], const float* ws,
+                                            int c0, float2 sa2) {
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
         const float4 w4 = *reinterpret_cast<const float4*>(ws + c0 + j);
@@ -101,45 +98,32 @@ __device__ __forceinline__ void fma_chunk32(float2 (&acc)[64], const uint32_t (&
     }
 }
 
-// The promotion of one scale group over this thread's 128 columns: four 32-column TMEM loads,
-// two in flight while the previous two are multiplied in.
-__device__ __forceinline__ void promote_fp32(float2 (&acc)[64], uint32_t taddr, const float* ws, float sa) {
+// The promotion of one scale group over this thread's 64 columns: two rounds of one 32-column
+// TMEM load, its wait, then the multiply-adds.
+__device__ __forceinline__ void promote_fp32(float2 (&acc)[kCols / 2], uint32_t taddr, const float* ws, float sa) {
     const float2 sa2 = make_float2(sa, sa);
-    uint32_t v[32], u[32];
-    MOE_TMEM_LD32(taddr, v);
-    MOE_TMEM_LD32(taddr + 32, u);
-    MOE_TMEM_WAIT_LD(v);
-    MOE_TMEM_WAIT_LD(u);
-    fma_chunk32(acc, v, ws, 0, sa2);
-    MOE_TMEM_LD32(taddr + 64, v);
-    fma_chunk32(acc, u, ws, 32, sa2);
-    MOE_TMEM_LD32(taddr + 96, u);
-    MOE_TMEM_WAIT_LD(v);
-    MOE_TMEM_WAIT_LD(u);
-    fma_chunk32(acc, v, ws, 64, sa2);
-    fma_chunk32(acc, u, ws, 96, sa2);
+#pragma unroll
+    for (int c = 0; c < kCols; c += 32) {
+        uint32_t v[32];
+        MOE_TMEM_LD32(taddr + c, v);
+        MOE_TMEM_WAIT_LD(v);
+        fma_chunk32(acc, v, ws, c, sa2);
+    }
 }
 
 // Same with UE8M0 scales: the scale is 2^(ea + ew - 254), exact.
-__device__ __forceinline__ void promote_mx(float2 (&acc2)[64], uint32_t taddr, const uint32_t* ws4, int ea,
+__device__ __forceinline__ void promote_mx(float2 (&acc2)[kCols / 2], uint32_t taddr, const uint32_t* ws4, int ea,
                                            int g) {
     float* acc = reinterpret_cast<float*>(acc2);
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-        uint32_t v[32], u[32];
-        MOE_TMEM_LD32(taddr + c * 64, v);
-        MOE_TMEM_LD32(taddr + c * 64 + 32, u);
+    for (int c = 0; c < kCols; c += 32) {
+        uint32_t v[32];
+        MOE_TMEM_LD32(taddr + c, v);
         MOE_TMEM_WAIT_LD(v);
-        MOE_TMEM_WAIT_LD(u);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-            const int ew = static_cast<int>((ws4[c * 64 + j] >> (8 * g)) & 0xFFu);
-            acc[c * 64 + j] = fmaf(__uint_as_float(v[j]), exp2_int(ea + ew - 254), acc[c * 64 + j]);
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int ew = static_cast<int>((ws4[c * 64 + 32 + j] >> (8 * g)) & 0xFFu);
-            acc[c * 64 + 32 + j] = fmaf(__uint_as_float(u[j]), exp2_int(ea + ew - 254), acc[c * 64 + 32 + j]);
+            const int ew = static_cast<int>((ws4[c + j] >> (8 * g)) & 0xFFu);
+            acc[c + j] = fmaf(__uint_as_float(v[j]), exp2_int(ea + ew - 254), acc[c + j]);
         }
     }
 }
@@ -276,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------------ epilogue
         const int ew = warp - kFirstEpiWarp;
         const int quad = warp & 3;                // TMEM lanes 32*quad .. 32*quad+31
-        const int half = ew >> 2;                 // columns half*128 .. half*128+127 of the tile
+        const int qtr = ew >> 2;                  // columns qtr*64 .. qtr*64+63 of the tile
         const int row_in_tile = quad * 32 + lane;
         uint32_t it = 0, kg = 0, tile = 0;
         bool ok = true;
@@ -289,9 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_ok = row_in_tile < cnt;
             const int r = row0 + row_in_tile;
 
-            float2 acc2[64];
+            float2 acc2[kCols / 2];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) acc2[i] = make_float2(0.0f, 0.0f);
+            for (int i = 0; i < kCols / 2; ++i) acc2[i] = make_float2(0.0f, 0.0f);
             float* acc = reinterpret_cast<float*>(acc2);
 
             for (int kb = 0; kb < KB && ok; ++kb, ++it) {
@@ -301,11 +285,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = false;
                     break;
                 }
-                const uint8_t* ws_stage = smem + L::sc + s * kScaleSlot + half * 128 * 4;
+                const uint8_t* ws_stage = smem + L::sc + s * kScaleSlot + qtr * kCols * 4;
                 const uint32_t saw = reinterpret_cast<const uint32_t*>(smem + L::sc + s * kScaleSlot + kWsBytes)
                     [(row0 & 3) + row_in_tile];
-                const float sa = __uint_as_float(saw);
-                const uint32_t sa4 = saw;
                 for (int g = 0; g < GPS; ++g, ++kg) {
                     const int b = kg & 1;
                     if (!mbar_wait(&tfull[b], (kg >> 1) & 1, abort_flag, p.status)) {
@@ -315,12 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     if (warp_active) {
                         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                               static_cast<uint32_t>(b * kTileN + half * 128);
+                                               static_cast<uint32_t>(b * kTileN + qtr * kCols);
                         if (RECIPE == 0)
-                            promote_fp32(acc2, taddr, reinterpret_cast<const float*>(ws_stage), sa);
+                            promote_fp32(acc2, taddr, reinterpret_cast<const float*>(ws_stage), __uint_as_float(saw));
                         else
                             promote_mx(acc2, taddr, reinterpret_cast<const uint32_t*>(ws_stage),
-                                       static_cast<int>((sa4 >> (8 * g)) & 0xFFu), g);
+                                       static_cast<int>((saw >> (8 * g)) & 0xFFu), g);
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -333,50 +315,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
 
             if (MODE == 0) {
-                // ---- SwiGLU + requantization: acc[0:64] gate, acc[64:128] up, act columns c0..c0+63
+                // ---- SwiGLU + requantization.  This quarter holds acc[0:32] gate and acc[32:64] up
+                // of act columns c0 .. c0+31 (the transform's 32-column interleave).
                 const int I = p.N >> 1;
-                const int c0 = nb * 128 + half * 64;
+                const int c0 = nb * 128 + qtr * 32;
                 if (warp_active) {
                     if (p.bias) {
-                        const uint4* bg = reinterpret_cast<const uint4*>(p.bias + static_cast<size_t>(e) * p.N + c0);
-                        const uint4* bu = reinterpret_cast<const uint4*>(p.bias + static_cast<size_t>(e) * p.N + I + c0);
-#pragma unroll
-                        for (int v = 0; v < 8; ++v) {
-                            const uint4 g4 = __ldg(bg + v), u4 = __ldg(bu + v);
-                            const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w}, uw[4] = {u4.x, u4.y, u4.z, u4.w};
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                acc[8 * v + 2 * q] += __uint_as_float(gw[q] << 16);
-                                acc[8 * v + 2 * q + 1] += __uint_as_float(gw[q] & 0xFFFF0000u);
-                                acc[64 + 8 * v + 2 * q] += __uint_as_float(uw[q] << 16);
-                                acc[64 + 8 * v + 2 * q + 1] += __uint_as_float(uw[q] & 0xFFFF0000u);
-                            }
-                        }
+                        add_bias32(acc, p.bias + static_cast<size_t>(e) * p.N + c0);
+                        add_bias32(acc + 32, p.bias + static_cast<size_t>(e) * p.N + I + c0);
                     }
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) {
-                        const float gt = acc[i], up = acc[64 + i];
+                    for (int i = 0; i < 32; ++i) {
+                        const float gt = acc[i], up = acc[32 + i];
                         acc[i] = __fdiv_rn(gt, 1.0f + expf(-gt)) * up;
                     }
                 }
-                if (RECIPE == 0) {
-                    float amax = 0.0f;
+                float amax = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(acc[i]));
+                for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(acc[i]));
+                if (RECIPE == 0) {
+                    // one 128-column group per row: combine the four quarters' maxima
                     const int buf = tile & 1;
-                    s_amax[(buf * 2 + half) * 128 + row_in_tile] = amax;
+                    s_amax[(buf * 4 + qtr) * 128 + row_in_tile] = amax;
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&amax_bar[buf]);
                     if (!mbar_wait(&amax_bar[buf], (tile >> 1) & 1, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
-                    amax = fmaxf(amax, s_amax[(buf * 2 + (half ^ 1)) * 128 + row_in_tile]);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) amax = fmaxf(amax, s_amax[(buf * 4 + q) * 128 + row_in_tile]);
                     const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
                     if (warp_active && row_ok) {
                         uint4* dst = reinterpret_cast<uint4*>(p.act_q + static_cast<size_t>(r) * I + c0);
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
+                        for (int w = 0; w < 2; ++w) {
                             uint4 q;
                             q.x = e4m3x4(__fdiv_rn(acc[16 * w + 0], sc), __fdiv_rn(acc[16 * w + 1], sc),
                                          __fdiv_rn(acc[16 * w + 2], sc), __fdiv_rn(acc[16 * w + 3], sc));
@@ -388,49 +361,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          __fdiv_rn(acc[16 * w + 14], sc), __fdiv_rn(acc[16 * w + 15], sc));
                             dst[w] = q;
                         }
-                        if (half == 0) static_cast<float*>(p.act_s)[static_cast<size_t>(nb) * p.a_pad + r] = sc;
+                        if (qtr == 0) static_cast<float*>(p.act_s)[static_cast<size_t>(nb) * p.a_pad + r] = sc;
                     }
                 } else if (warp_active && row_ok) {
-                    uint32_t* dst = reinterpret_cast<uint32_t*>(p.act_q + static_cast<size_t>(r) * I + c0);
+                    // MXFP8: these 32 act columns are exactly one scale group
+                    const int ex = mx_exponent(amax);
+                    const float inv = exp2_int(-ex);
+                    uint32_t q[8];
 #pragma unroll
-                    for (int grp = 0; grp < 2; ++grp) {
-                        float amax = 0.0f;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(acc[32 * grp + i]));
-                        const int ex = mx_exponent(amax);
-                        const float inv = exp2_int(-ex);
-                        uint32_t q[8];
-#pragma unroll
-                        for (int w = 0; w < 8; ++w)
-                            q[w] = e4m3x4(acc[32 * grp + 4 * w] * inv, acc[32 * grp + 4 * w + 1] * inv,
-                                          acc[32 * grp + 4 * w + 2] * inv, acc[32 * grp + 4 * w + 3] * inv);
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + 8 * grp);
-                        d4[0] = make_uint4(q[0], q[1], q[2], q[3]);
-                        d4[1] = make_uint4(q[4], q[5], q[6], q[7]);
-                        static_cast<uint8_t*>(p.act_s)[(static_cast<size_t>(nb) * p.a_pad + r) * 4 + half * 2 + grp] =
-                            static_cast<uint8_t>(ex + 127);
-                    }
+                    for (int w = 0; w < 8; ++w)
+                        q[w] = e4m3x4(acc[4 * w] * inv, acc[4 * w + 1] * inv, acc[4 * w + 2] * inv,
+                                      acc[4 * w + 3] * inv);
+                    uint4* d4 = reinterpret_cast<uint4*>(p.act_q + static_cast<size_t>(r) * I + c0);
+                    d4[0] = make_uint4(q[0], q[1], q[2], q[3]);
+                    d4[1] = make_uint4(q[4], q[5], q[6], q[7]);
+                    static_cast<uint8_t*>(p.act_s)[(static_cast<size_t>(nb) * p.a_pad + r) * 4 + qtr] =
+                        static_cast<uint8_t>(ex + 127);
                 }
             } else {
                 // ---- down projection: + bias, fp32 rows
-                const int c0 = nb * kTileN + half * 128;
+                const int c0 = nb * kTileN + qtr * kCols;
                 if (warp_active && row_ok && c0 < p.N) {
-                    float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.N + c0);
                     if (p.bias) {
-                        const uint4* bb = reinterpret_cast<const uint4*>(p.bias + static_cast<size_t>(e) * p.N + c0);
-#pragma unroll
-                        for (int v = 0; v < 16; ++v) {
-                            const uint4 b4 = __ldg(bb + v);
-                            const uint32_t bw[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                acc[8 * v + 2 * q] += __uint_as_float(bw[q] << 16);
-                                acc[8 * v + 2 * q + 1] += __uint_as_float(bw[q] & 0xFFFF0000u);
-                            }
-                        }
+                        add_bias32(acc, p.bias + static_cast<size_t>(e) * p.N + c0);
+                        add_bias32(acc + 32, p.bias + static_cast<size_t>(e) * p.N + c0 + 32);
                     }
+                    float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.N + c0);
 #pragma unroll
-                    for (int c = 0; c < 128; c += 4) dst[c >> 2] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                    for (int c = 0; c < kCols; c += 4)
+                        dst[c >> 2] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
                 }
             }
         }
@@ -453,7 +412,7 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, const CUtensorMap& tmA, cons
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, k_grouped_gemm<MODE, RECIPE>);
     if (e != cudaSuccess) return e;
-    if (fa.numRegs * kThreads < kRegsLow * 128 + kRegsHigh * 256) return cudaErrorInvalidConfiguration;
+    if (fa.numRegs * kThreads < kRegsLow * 128 + kRegsHigh * 512) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(k_grouped_gemm<MODE, RECIPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;

@@ -1,0 +1,34 @@
+// gemm_common.cuh -- pieces shared by the two grouped FP8 GEMM kernels (gemm.cu, gemm_narrow.cu).
+#pragma once
+
+#include "moe_common.cuh"
+#include "moe_kernels.h"
+
+namespace moe {
+
+constexpr unsigned long long kDrainLimitNs = 100000000ull;
+
+// Bounded wait used only while leaving after an abort: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, parity))
+        if (globaltimer_ns() - t0 > kDrainLimitNs) break;
+}
+
+// Add 32 bf16 bias values (16-byte aligned) to acc[0..31].
+__device__ __forceinline__ void add_bias32(float* acc, const __nv_bfloat16* bias) {
+    const uint4* b4 = reinterpret_cast<const uint4*>(bias);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const uint4 w = __ldg(b4 + v);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            acc[8 * v + 2 * q] += __uint_as_float(ww[q] << 16);
+            acc[8 * v + 2 * q + 1] += __uint_as_float(ww[q] & 0xFFFF0000u);
+        }
+    }
+}
+
+}  // namespace moe

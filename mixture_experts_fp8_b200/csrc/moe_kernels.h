@@ -84,14 +84,15 @@ cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtenso
 int set_last_error(int code, const char* msg);
 cudaError_t launch_selftest_wait(int32_t* status, uint32_t timeout_us, cudaStream_t s);
 
-// Column permutation applied to w13 by the transform: within each 256-column block nb,
-// [gate nb*128 + 0:64 | up nb*128 + 0:64 | gate nb*128 + 64:128 | up nb*128 + 64:128].
-// Returns the transformed row index of original column n (0 <= n < 2I).
+// Column permutation applied to w13 by the transform: within each 256-column block nb, four
+// 64-column quarters q = 0..3, each [gate nb*128 + 32q + 0:32 | up nb*128 + 32q + 0:32], so that
+// one GEMM epilogue thread holds matching gate and up columns.  Returns the transformed row index
+// of original column n (0 <= n < 2I).
 __host__ __device__ inline int w13_interleaved_row(int n, int I) {
     const int is_up = n >= I;
     const int i = is_up ? n - I : n;
     const int nb = i >> 7, within = i & 127;
-    return nb * 256 + (within >> 6) * 128 + is_up * 64 + (within & 63);
+    return nb * 256 + (within >> 5) * 64 + is_up * 32 + (within & 31);
 }
 
 }  // namespace moe

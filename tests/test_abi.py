@@ -90,6 +90,6 @@ def test_interleave_is_a_permutation():
     def row(n):
         up = n >= I
         i = n - I if up else n
-        return (i >> 7) * 256 + ((i & 127) >> 6) * 128 + up * 64 + (i & 63)
+        return (i >> 7) * 256 + ((i & 127) >> 5) * 64 + up * 32 + (i & 31)
     rows = sorted(row(n) for n in range(2 * I))
     assert rows == list(range(2 * I))
