@@ -81,6 +81,10 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s);
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         int num_sms, cudaStream_t s);
+cudaError_t launch_gemm_narrow(const GemmArgs& a, const CUtensorMap& tmW, const CUtensorMap& tmT,
+                               int num_sms, cudaStream_t s);
+// The narrow (swap-AB) GEMMs take problems averaging at most this many routed rows per expert.
+constexpr int kNarrowRowsPerExpert = 32;
 int set_last_error(int code, const char* msg);
 cudaError_t launch_selftest_wait(int32_t* status, uint32_t timeout_us, cudaStream_t s);
 

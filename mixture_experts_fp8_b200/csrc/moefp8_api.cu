@@ -314,10 +314,15 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     const int32_t* idx = topk_idx ? topk_idx : static_cast<const int32_t*>(at(L.topk_idx));
     const float* wts = topk_idx ? topk_weights : static_cast<const float*>(at(L.topk_weights));
 
+    // Few rows per expert (decode): the swap-AB kernels, weights as the M operand; else the wide
+    // kernels.  Both compute every row with the same operations, so the choice does not change bits.
+    const bool narrow = A <= moe::kNarrowRowsPerExpert * E;
     CUtensorMap tm_x, tm_w13, tm_act, tm_w2;
-    if ((rc = make_kmajor_map(&tm_x, at(L.xq), A, H, moe::kTileM))) return rc;
-    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(E) * 2 * I, H, moe::kTileN))) return rc;
-    if ((rc = make_kmajor_map(&tm_act, at(L.act_q), A, I, moe::kTileM))) return rc;
+    const uint32_t tok_box = narrow ? 16 : moe::kTileM;
+    if ((rc = make_kmajor_map(&tm_x, at(L.xq), A, H, tok_box))) return rc;
+    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(E) * 2 * I, H, narrow ? 32 : moe::kTileN)))
+        return rc;
+    if ((rc = make_kmajor_map(&tm_act, at(L.act_q), A, I, tok_box))) return rc;
     if ((rc = make_kmajor_map(&tm_w2, w2_t, static_cast<uint64_t>(E) * H, I, moe::kTileN))) return rc;
 
     cudaEvent_t* ev = nullptr;
@@ -361,7 +366,8 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     g1.act_q = static_cast<uint8_t*>(at(L.act_q));
     g1.act_s = at(L.act_s);
     g1.status = status;
-    MOE_CUDA_TRY(moe::launch_gemm(g1, tm_x, tm_w13, di.sms, s));
+    MOE_CUDA_TRY(narrow ? moe::launch_gemm_narrow(g1, tm_w13, tm_x, di.sms, s)
+                        : moe::launch_gemm(g1, tm_x, tm_w13, di.sms, s));
     MOE_CUDA_TRY(mark(4));
     moe::GemmArgs g2 = g1;
     g2.mode = 1;
@@ -373,7 +379,8 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     g2.act_q = nullptr;
     g2.act_s = nullptr;
     g2.out = static_cast<float*>(at(L.o));
-    MOE_CUDA_TRY(moe::launch_gemm(g2, tm_act, tm_w2, di.sms, s));
+    MOE_CUDA_TRY(narrow ? moe::launch_gemm_narrow(g2, tm_w2, tm_act, di.sms, s)
+                        : moe::launch_gemm(g2, tm_act, tm_w2, di.sms, s));
     MOE_CUDA_TRY(mark(5));
     moe::CombineArgs ca{static_cast<const float*>(at(L.o)), static_cast<const int32_t*>(at(L.row_of)), wts,
                         static_cast<__nv_bfloat16*>(y), T, H, K};

@@ -51,3 +51,22 @@ def test_given_routing_matches_computed():
     w = gp.ws_region("topk_weights", torch.float32, T * K).clone().view(T, K)
     y2 = bits(gp.forward(topk_idx=idx, topk_weights=w))
     assert np.array_equal(y1, y2)
+
+
+@pytest.mark.parametrize("recipe", [0, 1])
+def test_narrow_and_wide_kernels_agree_bit_for_bit(recipe):
+    """A batch with few rows per expert runs the swap-AB (narrow) GEMMs; the same tokens inside a
+    large batch run the wide GEMMs.  Both compute each row with the same operations, so the rows
+    must agree bit for bit (a row's output does not depend on the other rows)."""
+    from dataclasses import replace
+    base = replace(synth.SHAPES["decode"], recipe=recipe, biases=True)
+    small = synth.make_problem(base)                       # 64 tokens: 512 rows <= 32 * 128 -> narrow
+    big_shape = base.with_tokens(4096)                     # 32768 rows -> wide
+    x_big, logits_big, _ = synth.make_activations(big_shape)
+    assert torch.equal(x_big[:64], small.x) and torch.equal(logits_big[:64], small.logits)
+    gp = GpuProblem(small)
+    y_small = bits(gp.forward())
+    c = lib_cfg(big_shape)
+    ws = gp.moe.new_workspace(c)
+    y_big = bits(gp.forward(x=x_big.cuda(), logits=logits_big.cuda(), cfg=c, workspace=ws))
+    assert np.array_equal(y_small, y_big[:64])
