@@ -337,7 +337,9 @@ def main():
                     "frac": g1_tflops / fp8_peak}
         else:
             roof = {"bound": "hbm", "achieved": g1_gbs, "peak": hbm, "unit": "GB/s", "frac": g1_gbs / hbm}
-        roof.update({"kernel": "k_grouped_gemm<gate+up>", "traffic": traffic_for("gemm1", shape.name),
+        narrow = A <= 32 * shape.num_experts     # the library's rule for the swap-AB kernels
+        roof.update({"kernel": ("k_grouped_gemm_narrow" if narrow else "k_grouped_gemm") + "<gate+up>",
+                     "traffic": traffic_for("gemm1", shape.name),
                      "peak_source": f"{pk_kind} ({'sustained bf16 x2 for fp8' if compute_bound else 'copy'})",
                      "algorithmic_bytes_per_launch": g1_bytes, "ms_per_launch": g1_ms})
         layer_roof_s = max(fl / (fp8_peak * 1e12), alg / (hbm * 1e9))
