@@ -421,11 +421,8 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, const CUtensorMap& tmA, cons
 
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
                         cudaStream_t s) {
-    if (a.mode == 0) {
-        return a.recipe == 0 ? launch_gemm_t<0, 0>(a, tmA, tmB, num_sms, s)
-                             : launch_gemm_t<0, 1>(a, tmA, tmB, num_sms, s);
-    }
-    return a.recipe == 0 ? launch_gemm_t<1, 0>(a, tmA, tmB, num_sms, s) : launch_gemm_t<1, 1>(a, tmA, tmB, num_sms, s);
+    if (a.recipe != 0) return cudaErrorInvalidValue;   // MXFP8 runs gemm_mx.cu
+    return a.mode == 0 ? launch_gemm_t<0, 0>(a, tmA, tmB, num_sms, s) : launch_gemm_t<1, 0>(a, tmA, tmB, num_sms, s);
 }
 
 }  // namespace moe

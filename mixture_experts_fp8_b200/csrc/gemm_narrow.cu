@@ -397,12 +397,8 @@ static cudaError_t launch_narrow_t(const GemmArgs& a, const CUtensorMap& tmW, co
 
 cudaError_t launch_gemm_narrow(const GemmArgs& a, const CUtensorMap& tmW, const CUtensorMap& tmT, int num_sms,
                                cudaStream_t s) {
-    if (a.mode == 0) {
-        return a.recipe == 0 ? launch_narrow_t<0, 0>(a, tmW, tmT, num_sms, s)
-                             : launch_narrow_t<0, 1>(a, tmW, tmT, num_sms, s);
-    }
-    return a.recipe == 0 ? launch_narrow_t<1, 0>(a, tmW, tmT, num_sms, s)
-                         : launch_narrow_t<1, 1>(a, tmW, tmT, num_sms, s);
+    if (a.recipe != 0) return cudaErrorInvalidValue;   // MXFP8 runs gemm_mx.cu
+    return a.mode == 0 ? launch_narrow_t<0, 0>(a, tmW, tmT, num_sms, s) : launch_narrow_t<1, 0>(a, tmW, tmT, num_sms, s);
 }
 
 }  // namespace moe

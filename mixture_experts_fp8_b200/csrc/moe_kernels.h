@@ -66,7 +66,7 @@ struct GemmArgs {
     const int32_t* offsets;     // [E + 1]
     const int32_t* tile_start;  // [E + 1]
     const void* a_scale;        // [K/128][a_pad] 4-byte words: fp32, or 4 x UE8M0 (one per 32-block)
-    const void* w_scale;        // recipe 0: fp32 [E, K/128, N]; recipe 1: u8 [E, K/128, N, 4]
+    const void* w_scale;        // recipe 0: fp32 [E, K/128, N]; recipe 1: 512-byte atoms [E, N/128, K/128]
     const __nv_bfloat16* bias;  // [E, N] in the caller's column order, or null
     uint8_t* act_q;             // mode 0: [A, N/2]
     void* act_s;                // mode 0: [(N/2)/128][a_pad] 4-byte words
@@ -81,6 +81,8 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s);
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         int num_sms, cudaStream_t s);
+cudaError_t launch_gemm_mx(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
+                           cudaStream_t s);
 cudaError_t launch_gemm_narrow(const GemmArgs& a, const CUtensorMap& tmW, const CUtensorMap& tmT,
                                int num_sms, cudaStream_t s);
 // The narrow (swap-AB) GEMMs take problems averaging at most this many routed rows per expert.
@@ -97,6 +99,13 @@ __host__ __device__ inline int w13_interleaved_row(int n, int I) {
     const int i = is_up ? n - I : n;
     const int nb = i >> 7, within = i & 127;
     return nb * 256 + (within >> 5) * 64 + is_up * 32 + (within & 31);
+}
+
+// Its inverse: the original column of transformed row r.
+__host__ __device__ inline int w13_original_col(int r, int I) {
+    const int nb = r >> 8, q = (r & 255) >> 6, is_up = (r & 63) >> 5, i = r & 31;
+    const int act = nb * 128 + q * 32 + i;
+    return is_up ? I + act : act;
 }
 
 }  // namespace moe

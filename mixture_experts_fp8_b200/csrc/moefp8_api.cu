@@ -316,14 +316,19 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
 
     // Few rows per expert (decode): the swap-AB kernels, weights as the M operand; else the wide
     // kernels.  Both compute every row with the same operations, so the choice does not change bits.
-    const bool narrow = A <= moe::kNarrowRowsPerExpert * E;
+    // MXFP8 runs the block-scaled tensor-core kernels.  fp32 scales: few rows per expert (decode)
+    // take the swap-AB kernels, weights as the M operand, else the wide kernels; both compute every
+    // row with the same operations, so the choice does not change bits.
+    const bool mx = cfg->recipe == 1;
+    const bool narrow = !mx && A <= moe::kNarrowRowsPerExpert * E;
     CUtensorMap tm_x, tm_w13, tm_act, tm_w2;
     const uint32_t tok_box = narrow ? 16 : moe::kTileM;
+    const uint32_t w13_box = mx ? 128 : narrow ? 32 : moe::kTileN;
+    const uint32_t w2_box = mx ? 128 : moe::kTileN;
     if ((rc = make_kmajor_map(&tm_x, at(L.xq), A, H, tok_box))) return rc;
-    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(E) * 2 * I, H, narrow ? 32 : moe::kTileN)))
-        return rc;
+    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(E) * 2 * I, H, w13_box))) return rc;
     if ((rc = make_kmajor_map(&tm_act, at(L.act_q), A, I, tok_box))) return rc;
-    if ((rc = make_kmajor_map(&tm_w2, w2_t, static_cast<uint64_t>(E) * H, I, moe::kTileN))) return rc;
+    if ((rc = make_kmajor_map(&tm_w2, w2_t, static_cast<uint64_t>(E) * H, I, w2_box))) return rc;
 
     cudaEvent_t* ev = nullptr;
     if (prof && (rc = prof_next(prof, &ev))) return rc;
@@ -366,8 +371,9 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     g1.act_q = static_cast<uint8_t*>(at(L.act_q));
     g1.act_s = at(L.act_s);
     g1.status = status;
-    MOE_CUDA_TRY(narrow ? moe::launch_gemm_narrow(g1, tm_w13, tm_x, di.sms, s)
-                        : moe::launch_gemm(g1, tm_x, tm_w13, di.sms, s));
+    MOE_CUDA_TRY(mx       ? moe::launch_gemm_mx(g1, tm_x, tm_w13, di.sms, s)
+                 : narrow ? moe::launch_gemm_narrow(g1, tm_w13, tm_x, di.sms, s)
+                          : moe::launch_gemm(g1, tm_x, tm_w13, di.sms, s));
     MOE_CUDA_TRY(mark(4));
     moe::GemmArgs g2 = g1;
     g2.mode = 1;
@@ -379,8 +385,9 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     g2.act_q = nullptr;
     g2.act_s = nullptr;
     g2.out = static_cast<float*>(at(L.o));
-    MOE_CUDA_TRY(narrow ? moe::launch_gemm_narrow(g2, tm_w2, tm_act, di.sms, s)
-                        : moe::launch_gemm(g2, tm_act, tm_w2, di.sms, s));
+    MOE_CUDA_TRY(mx       ? moe::launch_gemm_mx(g2, tm_act, tm_w2, di.sms, s)
+                 : narrow ? moe::launch_gemm_narrow(g2, tm_w2, tm_act, di.sms, s)
+                          : moe::launch_gemm(g2, tm_act, tm_w2, di.sms, s));
     MOE_CUDA_TRY(mark(5));
     moe::CombineArgs ca{static_cast<const float*>(at(L.o)), static_cast<const int32_t*>(at(L.row_of)), wts,
                         static_cast<__nv_bfloat16*>(y), T, H, K};

@@ -107,8 +107,8 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
 // Weight transform (offline): E4M3 codes [E, K, N] -> K-major [E, N', K], with w13's columns
 // interleaved (moe::w13_interleaved_row), and the block scales re-laid to match:
 //   recipe 0: fp32 [E, K/128, N] -> [E, K/128, N'] (columns permuted like the codes)
-//   recipe 1: UE8M0 [E, K/32, N] -> [E, K/128, N', 4] (the four 32-deep blocks of each 128-deep
-//             stage packed into one 32-bit word per column)
+//   recipe 1: UE8M0 [E, K/32, N] -> 512-byte scale-factor atoms [E, N/128, K/128] for the
+//             block-scaled tensor core (see gemm_mx.cu)
 // ("MATE Mega MoE", transform_weights_for_mega_moe; "DeepGEMM PR #371", 4-packed UE8M0.)
 __global__ void __launch_bounds__(256) k_transpose_codes(const uint8_t* src, uint8_t* dst, int K,
                                                         int N, int interleave_I) {
@@ -134,23 +134,37 @@ __global__ void __launch_bounds__(256) k_transpose_codes(const uint8_t* src, uin
 
 __global__ void k_transform_scales(const void* src, void* dst, int E, int K, int N, int recipe,
                                    int interleave_I) {
-    const size_t total = static_cast<size_t>(E) * (K / 128) * N;
-    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const int n = static_cast<int>(i % N);
-        const size_t ek = i / N;                        // e * (K/128) + kb
-        const int row = interleave_I ? w13_interleaved_row(n, interleave_I) : n;
-        const size_t o = ek * N + row;
-        if (recipe == 0) {
-            static_cast<float*>(dst)[o] = static_cast<const float*>(src)[ek * N + n];
-        } else {
-            const size_t e = ek / (K / 128), kb = ek % (K / 128);
-            const uint8_t* s = static_cast<const uint8_t*>(src) + (e * (K / 32) + kb * 4) * N + n;
-            uint32_t w = static_cast<uint32_t>(s[0]) | (static_cast<uint32_t>(s[N]) << 8) |
-                         (static_cast<uint32_t>(s[2 * static_cast<size_t>(N)]) << 16) |
-                         (static_cast<uint32_t>(s[3 * static_cast<size_t>(N)]) << 24);
-            static_cast<uint32_t*>(dst)[o] = w;
+    if (recipe == 0) {
+        // fp32 [E, K/128, N] -> [E, K/128, N'] (columns permuted like the codes)
+        const size_t total = static_cast<size_t>(E) * (K / 128) * N;
+        for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+             i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+            const int n = static_cast<int>(i % N);
+            const size_t ek = i / N;                    // e * (K/128) + kb
+            const int row = interleave_I ? w13_interleaved_row(n, interleave_I) : n;
+            static_cast<float*>(dst)[ek * N + row] = static_cast<const float*>(src)[ek * N + n];
         }
+        return;
+    }
+    // UE8M0 [E, K/32, N] -> scale-factor atoms [E, N/128, K/128][512 B]: in the atom of column block
+    // nb and stage kb, byte 16*i + 4*c + k is the scale of transformed row nb*128 + 32*c + i for the
+    // 32-deep block kb*4 + k.
+    const int NB = N / 128, KB = K / 128;
+    const size_t total = static_cast<size_t>(E) * NB * KB * 512;
+    const uint8_t* s = static_cast<const uint8_t*>(src);
+    uint8_t* d = static_cast<uint8_t*>(dst);
+    for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const int byte = static_cast<int>(idx & 511);
+        const size_t atom = idx >> 9;                   // (e * NB + nb) * KB + kb
+        const int kb = static_cast<int>(atom % KB);
+        const size_t enb = atom / KB;
+        const int nb = static_cast<int>(enb % NB);
+        const size_t e = enb / NB;
+        const int i = byte >> 4, c = (byte >> 2) & 3, k = byte & 3;
+        const int row = nb * 128 + 32 * c + i;
+        const int col = interleave_I ? w13_original_col(row, interleave_I) : row;
+        d[idx] = s[(e * (K / 32) + kb * 4 + k) * N + col];
     }
 }
 
