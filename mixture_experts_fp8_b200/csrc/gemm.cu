@@ -1,5 +1,5 @@
-// gemm.cu -- grouped, block-scaled FP8 GEMM on the 5th-generation tensor cores (tcgen05), for
-// both expert projections of the layer.
+// gemm.cu -- grouped FP8 GEMM with fp32 block scales on the 5th-generation tensor cores
+// (tcgen05), for both expert projections of the layer (recipe 0; MXFP8 runs gemm_mx.cu).
 //
 //   mode 0 (gate+up): h[r, n] = sum_g a_s[r,g] * w_s[e,g,n] * sum_{k in g} xq[r,k] * w13[e,n,k]
 //                     (+ b13), then act = silu(h_gate) * h_up, requantized per (row, g)
@@ -13,9 +13,8 @@
 //   warp 0   TMA producer: per 128-deep K stage, a 128x128 A tile and a 256x128 B tile (both
 //            K-major, 128-byte swizzle), the 256 weight scales of the stage and the tile rows'
 //            activation scales (bulk copies).
-//   warp 1   MMA issuer (one thread): tcgen05.mma.kind::f8f6f4, M=128 N=256 K=32.  Each scale
-//            group (128 deep for recipe 0, 32 for recipe 1) is accumulated alone into one of two
-//            256-column fp32 TMEM buffers.
+//   warp 1   MMA issuer (one thread): tcgen05.mma.kind::f8f6f4, M=128 N=256 K=32.  Each 128-deep
+//            scale group is accumulated alone into one of two 256-column fp32 TMEM buffers.
 //   warps 2-3 idle.  Warpgroup 0 gives registers back (setmaxnreg.dec to 32).
 //   warps 4-19 epilogue (setmaxnreg.inc to 112): warp w reads TMEM lanes 32*(w%4) .. +31 (tile
 //            rows) and one quarter of the columns; every group partial is multiplied by
@@ -111,26 +110,9 @@ __device__ __forceinline__ void promote_fp32(float2 (&acc)[kCols / 2], uint32_t 
     }
 }
 
-// Same with UE8M0 scales: the scale is 2^(ea + ew - 254), exact.
-__device__ __forceinline__ void promote_mx(float2 (&acc2)[kCols / 2], uint32_t taddr, const uint32_t* ws4, int ea,
-                                           int g) {
-    float* acc = reinterpret_cast<float*>(acc2);
-#pragma unroll
-    for (int c = 0; c < kCols; c += 32) {
-        uint32_t v[32];
-        MOE_TMEM_LD32(taddr + c, v);
-        MOE_TMEM_WAIT_LD(v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int ew = static_cast<int>((ws4[c + j] >> (8 * g)) & 0xFFu);
-            acc[c + j] = fmaf(__uint_as_float(v[j]), exp2_int(ea + ew - 254), acc[c + j]);
-        }
-    }
-}
-
 }  // namespace
 
-template <int MODE, int RECIPE>
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_grouped_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const GemmArgs p) {
@@ -181,8 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_holder;
     const int total_units = s_tstart[p.E] * nt;
     const int KB = p.K / kTileK;                 // pipeline stages per unit
-    constexpr int GPS = RECIPE == 0 ? 1 : 4;     // scale groups per stage
-    constexpr int MPG = 4 / GPS;                 // K=32 MMAs per scale group
+    constexpr int GPS = 1;                       // scale groups per stage
+    constexpr int MPG = 4;                       // K=32 MMAs per scale group
 
     if (warp < kFirstEpiWarp) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
@@ -298,11 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (warp_active) {
                         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                                static_cast<uint32_t>(b * kTileN + qtr * kCols);
-                        if (RECIPE == 0)
-                            promote_fp32(acc2, taddr, reinterpret_cast<const float*>(ws_stage), __uint_as_float(saw));
-                        else
-                            promote_mx(acc2, taddr, reinterpret_cast<const uint32_t*>(ws_stage),
-                                       static_cast<int>((saw >> (8 * g)) & 0xFFu), g);
+                        promote_fp32(acc2, taddr, reinterpret_cast<const float*>(ws_stage), __uint_as_float(saw));
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -333,50 +311,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float amax = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(acc[i]));
-                if (RECIPE == 0) {
-                    // one 128-column group per row: combine the four quarters' maxima
-                    const int buf = tile & 1;
-                    s_amax[(buf * 4 + qtr) * 128 + row_in_tile] = amax;
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&amax_bar[buf]);
-                    if (!mbar_wait(&amax_bar[buf], (tile >> 1) & 1, abort_flag, p.status)) {
-                        ok = false;
-                        break;
+                // one 128-column group per row: combine the four quarters' maxima
+                const int buf = tile & 1;
+                s_amax[(buf * 4 + qtr) * 128 + row_in_tile] = amax;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&amax_bar[buf]);
+                if (!mbar_wait(&amax_bar[buf], (tile >> 1) & 1, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) amax = fmaxf(amax, s_amax[(buf * 4 + q) * 128 + row_in_tile]);
+                const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+                if (warp_active && row_ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.act_q + static_cast<size_t>(r) * I + c0);
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        uint4 q;
+                        q.x = e4m3x4(__fdiv_rn(acc[16 * w + 0], sc), __fdiv_rn(acc[16 * w + 1], sc),
+                                     __fdiv_rn(acc[16 * w + 2], sc), __fdiv_rn(acc[16 * w + 3], sc));
+                        q.y = e4m3x4(__fdiv_rn(acc[16 * w + 4], sc), __fdiv_rn(acc[16 * w + 5], sc),
+                                     __fdiv_rn(acc[16 * w + 6], sc), __fdiv_rn(acc[16 * w + 7], sc));
+                        q.z = e4m3x4(__fdiv_rn(acc[16 * w + 8], sc), __fdiv_rn(acc[16 * w + 9], sc),
+                                     __fdiv_rn(acc[16 * w + 10], sc), __fdiv_rn(acc[16 * w + 11], sc));
+                        q.w = e4m3x4(__fdiv_rn(acc[16 * w + 12], sc), __fdiv_rn(acc[16 * w + 13], sc),
+                                     __fdiv_rn(acc[16 * w + 14], sc), __fdiv_rn(acc[16 * w + 15], sc));
+                        dst[w] = q;
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) amax = fmaxf(amax, s_amax[(buf * 4 + q) * 128 + row_in_tile]);
-                    const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-                    if (warp_active && row_ok) {
-                        uint4* dst = reinterpret_cast<uint4*>(p.act_q + static_cast<size_t>(r) * I + c0);
-#pragma unroll
-                        for (int w = 0; w < 2; ++w) {
-                            uint4 q;
-                            q.x = e4m3x4(__fdiv_rn(acc[16 * w + 0], sc), __fdiv_rn(acc[16 * w + 1], sc),
-                                         __fdiv_rn(acc[16 * w + 2], sc), __fdiv_rn(acc[16 * w + 3], sc));
-                            q.y = e4m3x4(__fdiv_rn(acc[16 * w + 4], sc), __fdiv_rn(acc[16 * w + 5], sc),
-                                         __fdiv_rn(acc[16 * w + 6], sc), __fdiv_rn(acc[16 * w + 7], sc));
-                            q.z = e4m3x4(__fdiv_rn(acc[16 * w + 8], sc), __fdiv_rn(acc[16 * w + 9], sc),
-                                         __fdiv_rn(acc[16 * w + 10], sc), __fdiv_rn(acc[16 * w + 11], sc));
-                            q.w = e4m3x4(__fdiv_rn(acc[16 * w + 12], sc), __fdiv_rn(acc[16 * w + 13], sc),
-                                         __fdiv_rn(acc[16 * w + 14], sc), __fdiv_rn(acc[16 * w + 15], sc));
-                            dst[w] = q;
-                        }
-                        if (qtr == 0) static_cast<float*>(p.act_s)[static_cast<size_t>(nb) * p.a_pad + r] = sc;
-                    }
-                } else if (warp_active && row_ok) {
-                    // MXFP8: these 32 act columns are exactly one scale group
-                    const int ex = mx_exponent(amax);
-                    const float inv = exp2_int(-ex);
-                    uint32_t q[8];
-#pragma unroll
-                    for (int w = 0; w < 8; ++w)
-                        q[w] = e4m3x4(acc[4 * w] * inv, acc[4 * w + 1] * inv, acc[4 * w + 2] * inv,
-                                      acc[4 * w + 3] * inv);
-                    uint4* d4 = reinterpret_cast<uint4*>(p.act_q + static_cast<size_t>(r) * I + c0);
-                    d4[0] = make_uint4(q[0], q[1], q[2], q[3]);
-                    d4[1] = make_uint4(q[4], q[5], q[6], q[7]);
-                    static_cast<uint8_t*>(p.act_s)[(static_cast<size_t>(nb) * p.a_pad + r) * 4 + qtr] =
-                        static_cast<uint8_t>(ex + 127);
+                    if (qtr == 0) static_cast<float*>(p.act_s)[static_cast<size_t>(nb) * p.a_pad + r] = sc;
                 }
             } else {
                 // ---- down projection: + bias, fp32 rows
@@ -404,25 +366,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int MODE, int RECIPE>
+template <int MODE>
 static cudaError_t launch_gemm_t(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
                                  cudaStream_t s) {
     // The register split above must fit what the block is launched with, or setmaxnreg.inc
     // would wait forever: refuse to launch otherwise.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, k_grouped_gemm<MODE, RECIPE>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, k_grouped_gemm<MODE>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs * kThreads < kRegsLow * 128 + kRegsHigh * 512) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(k_grouped_gemm<MODE, RECIPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_grouped_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
-    return launch_pdl(k_grouped_gemm<MODE, RECIPE>, dim3(num_sms), dim3(kThreads), kSmemBytes, s, tmA, tmB, a);
+    return launch_pdl(k_grouped_gemm<MODE>, dim3(num_sms), dim3(kThreads), kSmemBytes, s, tmA, tmB, a);
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
                         cudaStream_t s) {
     if (a.recipe != 0) return cudaErrorInvalidValue;   // MXFP8 runs gemm_mx.cu
-    return a.mode == 0 ? launch_gemm_t<0, 0>(a, tmA, tmB, num_sms, s) : launch_gemm_t<1, 0>(a, tmA, tmB, num_sms, s);
+    return a.mode == 0 ? launch_gemm_t<0>(a, tmA, tmB, num_sms, s) : launch_gemm_t<1>(a, tmA, tmB, num_sms, s);
 }
 
 }  // namespace moe

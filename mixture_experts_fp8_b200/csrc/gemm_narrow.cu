@@ -1,6 +1,6 @@
-// gemm_narrow.cu -- the grouped, block-scaled FP8 GEMMs for problems with few routed rows per
-// expert (decode), in the swap-AB orientation: the expert's weights are the MMA's M=128 operand
-// and its routed rows (tokens) the N=16 operand.
+// gemm_narrow.cu -- the grouped FP8 GEMMs with fp32 block scales (recipe 0) for problems with few
+// routed rows per expert (decode), in the swap-AB orientation: the expert's weights are the MMA's
+// M=128 operand and its routed rows (tokens) the N=16 operand.
 //
 // Same arithmetic as gemm.cu, term for term ("metrale_model_layers fp8_grouped_tc_w8a8.rs",
 // run_fp8_grouped_w8a8; "MATE Mega MoE", API: swiglu):
@@ -78,7 +78,7 @@ __device__ __forceinline__ void decode_unit_narrow(int u, const int* ustart, con
 
 }  // namespace
 
-template <int MODE, int RECIPE>
+template <int MODE>
 __global__ void __launch_bounds__(kNThreads, 1)
     k_grouped_gemm_narrow(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
                           const GemmArgs p) {
@@ -138,8 +138,8 @@ __global__ void __launch_bounds__(kNThreads, 1)
     const uint32_t tmem_base = *tmem_holder;
     const int total_units = s_ustart[p.E];
     const int KB = p.K / kTileK;
-    constexpr int GPS = RECIPE == 0 ? 1 : 4;
-    constexpr int MPG = 4 / GPS;
+    constexpr int GPS = 1;                       // one 128-deep scale group per stage
+    constexpr int MPG = 4;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -263,23 +263,12 @@ __global__ void __launch_bounds__(kNThreads, 1)
                     MOE_TMEM_LD16(taddr + kNT, v1);
                     MOE_TMEM_WAIT_LD16(v0);
                     MOE_TMEM_WAIT_LD16(v1);
-                    if (RECIPE == 0) {
-                        const float ws0 = __uint_as_float(w0), ws1 = __uint_as_float(w1);
+                    const float ws0 = __uint_as_float(w0), ws1 = __uint_as_float(w1);
 #pragma unroll
-                        for (int t = 0; t < kNT; ++t) {
-                            const float sa = __uint_as_float(saw[t]);
-                            acc0[t] = fmaf(__uint_as_float(v0[t]), ws0 * sa, acc0[t]);
-                            acc1[t] = fmaf(__uint_as_float(v1[t]), ws1 * sa, acc1[t]);
-                        }
-                    } else {
-                        const int e0 = static_cast<int>((w0 >> (8 * g)) & 0xFFu) - 254;
-                        const int e1 = static_cast<int>((w1 >> (8 * g)) & 0xFFu) - 254;
-#pragma unroll
-                        for (int t = 0; t < kNT; ++t) {
-                            const int ea = static_cast<int>((saw[t] >> (8 * g)) & 0xFFu);
-                            acc0[t] = fmaf(__uint_as_float(v0[t]), exp2_int(ea + e0), acc0[t]);
-                            acc1[t] = fmaf(__uint_as_float(v1[t]), exp2_int(ea + e1), acc1[t]);
-                        }
+                    for (int t = 0; t < kNT; ++t) {
+                        const float sa = __uint_as_float(saw[t]);
+                        acc0[t] = fmaf(__uint_as_float(v0[t]), ws0 * sa, acc0[t]);
+                        acc1[t] = fmaf(__uint_as_float(v1[t]), ws1 * sa, acc1[t]);
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -305,56 +294,40 @@ __global__ void __launch_bounds__(kNThreads, 1)
                 }
 #pragma unroll
                 for (int t = 0; t < kNT; ++t) acc0[t] = __fdiv_rn(acc0[t], 1.0f + expf(-acc0[t])) * acc1[t];
-                if (RECIPE == 0) {
-                    // per token, the maximum over the 128 act columns of this tile (four warps)
-                    const int buf = tile & 1;
-                    if (tile >= 2 && !mbar_wait(&amax_free[buf], ((tile >> 1) + 1) & 1, abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
+                // per token, the maximum over the 128 act columns of this tile (four warps)
+                const int buf = tile & 1;
+                if (tile >= 2 && !mbar_wait(&amax_free[buf], ((tile >> 1) + 1) & 1, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
 #pragma unroll
-                    for (int t = 0; t < kNT; ++t) {
-                        const float m = warp_max(fabsf(acc0[t]));
-                        if (lane == t) s_amax[(buf * 4 + quad) * kNT + t] = m;
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&amax_bar[buf]);
-                    if (!mbar_wait(&amax_bar[buf], (tile >> 1) & 1, abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    float sc[kNT];
+                for (int t = 0; t < kNT; ++t) {
+                    const float m = warp_max(fabsf(acc0[t]));
+                    if (lane == t) s_amax[(buf * 4 + quad) * kNT + t] = m;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&amax_bar[buf]);
+                if (!mbar_wait(&amax_bar[buf], (tile >> 1) & 1, abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                float sc[kNT];
 #pragma unroll
-                    for (int t = 0; t < kNT; ++t) {
-                        float m = s_amax[(buf * 4 + 0) * kNT + t];
+                for (int t = 0; t < kNT; ++t) {
+                    float m = s_amax[(buf * 4 + 0) * kNT + t];
 #pragma unroll
-                        for (int q = 1; q < 4; ++q) m = fmaxf(m, s_amax[(buf * 4 + q) * kNT + t]);
-                        sc[t] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&amax_free[buf]);
+                    for (int q = 1; q < 4; ++q) m = fmaxf(m, s_amax[(buf * 4 + q) * kNT + t]);
+                    sc[t] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&amax_free[buf]);
 #pragma unroll
-                    for (int t = 0; t < kNT; ++t) {
-                        if (t < cnt) {
-                            const size_t r = static_cast<size_t>(row0 + t);
-                            p.act_q[r * I + c] = static_cast<uint8_t>(e4m3x2(__fdiv_rn(acc0[t], sc[t]), 0.0f) & 0xFFu);
-                            if (quad == 0 && lane == 0)
-                                static_cast<float*>(p.act_s)[static_cast<size_t>(wb) * p.a_pad + r] = sc[t];
-                        }
-                    }
-                } else {
-                    // MXFP8: the 32 act columns of this warp are one scale group
-#pragma unroll
-                    for (int t = 0; t < kNT; ++t) {
-                        const float m = warp_max(fabsf(acc0[t]));
-                        const int ex = mx_exponent(m);
-                        if (t < cnt) {
-                            const size_t r = static_cast<size_t>(row0 + t);
-                            p.act_q[r * I + c] = static_cast<uint8_t>(e4m3x2(acc0[t] * exp2_int(-ex), 0.0f) & 0xFFu);
-                            if (lane == 0)
-                                static_cast<uint8_t*>(p.act_s)[(static_cast<size_t>(wb) * p.a_pad + r) * 4 + quad] =
-                                    static_cast<uint8_t>(ex + 127);
-                        }
+                for (int t = 0; t < kNT; ++t) {
+                    if (t < cnt) {
+                        const size_t r = static_cast<size_t>(row0 + t);
+                        p.act_q[r * I + c] = static_cast<uint8_t>(e4m3x2(__fdiv_rn(acc0[t], sc[t]), 0.0f) & 0xFFu);
+                        if (quad == 0 && lane == 0)
+                            static_cast<float*>(p.act_s)[static_cast<size_t>(wb) * p.a_pad + r] = sc[t];
                     }
                 }
             } else {
@@ -385,20 +358,20 @@ __global__ void __launch_bounds__(kNThreads, 1)
     }
 }
 
-template <int MODE, int RECIPE>
+template <int MODE>
 static cudaError_t launch_narrow_t(const GemmArgs& a, const CUtensorMap& tmW, const CUtensorMap& tmT, int num_sms,
                                    cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_narrow<MODE, RECIPE>,
+    cudaError_t e = cudaFuncSetAttribute(k_grouped_gemm_narrow<MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kNSmemBytes));
     if (e != cudaSuccess) return e;
-    return launch_pdl(k_grouped_gemm_narrow<MODE, RECIPE>, dim3(num_sms), dim3(kNThreads), kNSmemBytes, s, tmW,
+    return launch_pdl(k_grouped_gemm_narrow<MODE>, dim3(num_sms), dim3(kNThreads), kNSmemBytes, s, tmW,
                       tmT, a);
 }
 
 cudaError_t launch_gemm_narrow(const GemmArgs& a, const CUtensorMap& tmW, const CUtensorMap& tmT, int num_sms,
                                cudaStream_t s) {
     if (a.recipe != 0) return cudaErrorInvalidValue;   // MXFP8 runs gemm_mx.cu
-    return a.mode == 0 ? launch_narrow_t<0, 0>(a, tmW, tmT, num_sms, s) : launch_narrow_t<1, 0>(a, tmW, tmT, num_sms, s);
+    return a.mode == 0 ? launch_narrow_t<0>(a, tmW, tmT, num_sms, s) : launch_narrow_t<1>(a, tmW, tmT, num_sms, s);
 }
 
 }  // namespace moe

@@ -9,6 +9,7 @@
 namespace moe {
 
 constexpr int kPermuteChunk = 256;    // routed rows per histogram / scatter chunk
+constexpr int kSmallRows = 2048;      // batches up to this many routed rows are permuted by one block
 constexpr int kTileM = 128;           // GEMM rows per tile
 constexpr int kTileN = 256;           // GEMM output columns per tile
 constexpr int kTileK = 128;           // K bytes (= E4M3 elements) per pipeline stage
@@ -20,6 +21,7 @@ struct RouteArgs {
     float* w;                   // [T, K]
     int T, E, K, routing, renorm, G, kg, mode;
     float rsf;
+    int32_t* status;            // cleared to MOE_OK by the first thread when non-null
 };
 
 struct PermuteArgs {
@@ -76,6 +78,7 @@ struct GemmArgs {
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
+cudaError_t launch_permute_small(const PermuteArgs& pa, bool clear_status, cudaStream_t s);
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s);

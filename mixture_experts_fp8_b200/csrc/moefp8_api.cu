@@ -275,7 +275,7 @@ int moe_route(const moe_config_t* cfg, const float* router_logits, const float* 
     if ((rc = device_info(&di))) return rc;
     moe::RouteArgs a{router_logits, per_expert_scale, topk_idx, topk_weights, cfg->num_tokens, cfg->num_experts,
                      cfg->top_k, cfg->routing, cfg->renormalize, cfg->group_count, cfg->k_group,
-                     cfg->group_select_mode, cfg->routed_scaling_factor};
+                     cfg->group_select_mode, cfg->routed_scaling_factor, nullptr};
     MOE_CUDA_TRY(moe::launch_route(a, static_cast<cudaStream_t>(stream)));
     return ok();
 }
@@ -335,20 +335,26 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     cudaStream_t s = static_cast<cudaStream_t>(stream_);
     auto mark = [&](int i) -> cudaError_t { return ev ? cudaEventRecord(ev[i], s) : cudaSuccess; };
 
-    MOE_CUDA_TRY(mark(0));
-    MOE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
-    if (router_logits) {
-        moe::RouteArgs ra{router_logits, per_expert_scale, static_cast<int32_t*>(at(L.topk_idx)),
-                          static_cast<float*>(at(L.topk_weights)), T, E, K, cfg->routing, cfg->renormalize,
-                          cfg->group_count, cfg->k_group, cfg->group_select_mode, cfg->routed_scaling_factor};
-        MOE_CUDA_TRY(moe::launch_route(ra, s));
-    }
-    MOE_CUDA_TRY(mark(1));
+    moe::RouteArgs ra{router_logits, per_expert_scale, static_cast<int32_t*>(at(L.topk_idx)),
+                      static_cast<float*>(at(L.topk_weights)), T, E, K, cfg->routing, cfg->renormalize,
+                      cfg->group_count, cfg->k_group, cfg->group_select_mode, cfg->routed_scaling_factor,
+                      nullptr};
     moe::PermuteArgs pa{idx, static_cast<int32_t*>(at(L.hist)), static_cast<int32_t*>(at(L.counts)),
                         static_cast<int32_t*>(at(L.offsets)), static_cast<int32_t*>(at(L.tile_start)),
                         static_cast<int32_t*>(at(L.row_src)), static_cast<int32_t*>(at(L.row_of)), expert_counts,
                         status, A, E, (A + moe::kPermuteChunk - 1) / moe::kPermuteChunk};
-    MOE_CUDA_TRY(moe::launch_permute(pa, s));
+    MOE_CUDA_TRY(mark(0));
+    // The first kernel of the forward clears the status word: the router when it runs, else the
+    // small-batch permutation; a memset otherwise.
+    if (router_logits) {
+        ra.status = status;
+        MOE_CUDA_TRY(moe::launch_route(ra, s));
+    } else if (A > moe::kSmallRows) {
+        MOE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    }
+    MOE_CUDA_TRY(mark(1));
+    if (A <= moe::kSmallRows) MOE_CUDA_TRY(moe::launch_permute_small(pa, router_logits == nullptr, s));
+    else MOE_CUDA_TRY(moe::launch_permute(pa, s));
     MOE_CUDA_TRY(mark(2));
     moe::QuantArgs qa{static_cast<const __nv_bfloat16*>(hidden_states), static_cast<const int32_t*>(at(L.row_of)),
                       static_cast<uint8_t*>(at(L.xq)), at(L.xs), status, T, H, K, cfg->recipe,

@@ -125,6 +125,120 @@ __global__ void __launch_bounds__(32) k_scatter(PermuteArgs a) {
     }
 }
 
+// ------------------------------------------------------------------------------------------
+// Small batches (A <= kSmallRows): one block does what the three kernels above do, with the same
+// result: per-warp histograms over 16 contiguous chunks of routed rows, per-expert bases across
+// chunks, counts / offsets / tile starts, then each warp scatters its chunk in row order.
+constexpr int kSmallWarps = 16;
+constexpr size_t kSmallSmem = kSmallRows * 4 + kSmallWarps * MOE_MAX_EXPERTS * 4 + MOE_MAX_EXPERTS * 4;
+
+__global__ void __launch_bounds__(kSmallWarps * 32) k_permute_small(PermuteArgs pa, int clear_status) {
+    extern __shared__ uint8_t sm[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int* ids = reinterpret_cast<int*>(sm);
+    int* hist = ids + kSmallRows;                      // [warp][E]
+    int* off_s = hist + kSmallWarps * MOE_MAX_EXPERTS;
+    const int A = pa.A, E = pa.E;
+    pdl_wait_then_release();
+    if (clear_status && threadIdx.x == 0 && pa.status) *pa.status = MOE_OK;
+    for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) hist[i] = 0;
+    for (int r = threadIdx.x; r < A; r += blockDim.x) ids[r] = pa.idx[r];
+    __syncthreads();
+    const int C = ((A + kSmallWarps - 1) / kSmallWarps + 31) / 32 * 32;
+    const int begin = warp * C, end = min(A, begin + C);
+    for (int r = begin + lane; r < end; r += 32) {
+        const int e = ids[r];
+        if (e >= 0 && e < E) atomicAdd(&hist[warp * E + e], 1);
+        else set_status(pa.status, MOE_ERR_BOUNDS);
+    }
+    __syncthreads();
+    if (threadIdx.x < E) {                             // bases across chunks, totals
+        const int e = threadIdx.x;
+        int run = 0;
+        for (int w = 0; w < kSmallWarps; ++w) {
+            const int v = hist[w * E + e];
+            hist[w * E + e] = run;
+            run += v;
+        }
+        off_s[e] = run;
+    }
+    __syncthreads();
+    if (warp == 0) {                                   // scans over experts: lane l owns 8l .. 8l+7
+        int c[8], mt[8], sc = 0, sm_ = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            c[i] = e < E ? off_s[e] : 0;
+            mt[i] = (c[i] + kTileM - 1) / kTileM;
+            sc += c[i];
+            sm_ += mt[i];
+        }
+        int xc = sc, xm = sm_;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int yc = __shfl_up_sync(0xffffffffu, xc, o), ym = __shfl_up_sync(0xffffffffu, xm, o);
+            if (lane >= o) {
+                xc += yc;
+                xm += ym;
+            }
+        }
+        int base = xc - sc, mbase = xm - sm_;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane * 8 + i;
+            if (e < E) {
+                pa.counts[e] = c[i];
+                pa.offsets[e] = base;
+                pa.tile_start[e] = mbase;
+                if (pa.expert_counts) pa.expert_counts[e] = c[i];
+                off_s[e] = base;
+            }
+            base += c[i];
+            mbase += mt[i];
+        }
+        if (lane == 31) {
+            pa.offsets[E] = base;
+            pa.tile_start[E] = mbase;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) hist[i] += off_s[i % E];
+    __syncthreads();
+    for (int r0 = begin; r0 < end; r0 += 32) {         // stable scatter of this warp's chunk
+        const int r = r0 + lane;
+        const bool valid = r < end;
+        int e = valid ? ids[r] : -1;
+        if (e >= E) e = -1;
+        const uint32_t active = __ballot_sync(0xffffffffu, valid && e >= 0);
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        const uint32_t mine = peers & active;
+        const int rank = __popc(mine & ((1u << lane) - 1u));
+        int dst = 0;
+        if (valid && e >= 0) dst = hist[warp * E + e] + rank;
+        __syncwarp();
+        if (valid && e >= 0 && rank == 0) hist[warp * E + e] += __popc(mine);
+        __syncwarp();
+        if (valid && e >= 0) {
+            pa.row_src[dst] = r;
+            pa.row_of[r] = dst;
+        }
+    }
+}
+
+cudaError_t launch_permute_small(const PermuteArgs& pa, bool clear_status, cudaStream_t s) {
+    static bool configured[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64 && !configured[dev]) {
+        e = cudaFuncSetAttribute(k_permute_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kSmallSmem));
+        if (e != cudaSuccess) return e;
+        configured[dev] = true;
+    }
+    return launch_pdl(k_permute_small, dim3(1), dim3(kSmallWarps * 32), kSmallSmem, s, pa, clear_status ? 1 : 0);
+}
+
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s) {
     cudaError_t e = launch_pdl(k_hist, dim3(a.chunks), dim3(256), 0, s, a);
     if (e == cudaSuccess) e = launch_pdl(k_scan, dim3(1), dim3(256), 0, s, a);

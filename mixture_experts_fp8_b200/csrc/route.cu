@@ -1,36 +1,10 @@
-// route.cu -- router top-k: one warp per token.
-//
-// "MindIE-SD Fused MoE", routing selection and parameter table: softmax or sigmoid scores,
-// optional expert-group pre-selection (group score = max, or sum of the two largest), top_k
-// inside the kept groups, renormalize (softmax), normalized weights (sigmoid),
-// routed_scaling_factor applied at selection.  "mlx_native ops/moe_gate.rs": top-K, softmax,
-// per_expert_scale, ids u32/int and fp32 weights [T, k].
-//
-// Experts are ranked by their raw logits (softmax and sigmoid are monotone), ties to the lower
-// index; group scores are fp32 scores, ties to the lower group.  Lane l holds experts
-// l, l+32, ... (E <= 256 -> at most 8 per lane); each top-k round is a warp arg-max over
-// (value desc, index asc) keys.
-#include <math.h>
-
-#include "moe_common.cuh"
-#include "moe_kernels.h"
+// route.cu -- the router top-k kernel (moe_route, and the first stage of large batches):
+// one warp per token; the per-token work is route_token() in route_device.cuh.
+#include "route_device.cuh"
 
 namespace moe {
 
 constexpr int kRouteWarps = 4;
-
-// Keep the better of (v, i) and the partner lanes' keys; i < 0 marks "none".
-__device__ __forceinline__ void argmax_reduce(float& v, int& i) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        float ov = __shfl_xor_sync(0xffffffffu, v, o);
-        int oi = __shfl_xor_sync(0xffffffffu, i, o);
-        if (oi >= 0 && (i < 0 || ov > v || (ov == v && oi < i))) {
-            v = ov;
-            i = oi;
-        }
-    }
-}
 
 __global__ void __launch_bounds__(kRouteWarps * 32) k_route(RouteArgs a) {
     __shared__ float s_score[kRouteWarps][256];
@@ -39,128 +13,11 @@ __global__ void __launch_bounds__(kRouteWarps * 32) k_route(RouteArgs a) {
     __shared__ unsigned char s_elig[kRouteWarps][256];
 
     pdl_wait_then_release();
+    if (a.status && blockIdx.x == 0 && threadIdx.x == 0) *a.status = MOE_OK;   // first kernel of a forward
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * kRouteWarps + warp;
     if (t >= a.T) return;
-    const int E = a.E;
-    const float* l = a.logits + static_cast<size_t>(t) * E;
-
-    float lv[8];
-    uint32_t okmask = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int e = lane + 32 * i;
-        lv[i] = -INFINITY;
-        if (e < E) {
-            lv[i] = l[e];
-            okmask |= 1u << i;
-        }
-    }
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if (okmask >> i & 1) m = fmaxf(m, lv[i]);
-    m = warp_max(m);
-    float z = 0.0f;
-    if (a.routing == 0) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (okmask >> i & 1) z += expf(lv[i] - m);
-        z = warp_sum(z);
-    }
-
-    // ---- expert-group pre-selection
-    if (a.G > 1) {
-        const int G = a.G, gs = E / G;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (okmask >> i & 1)
-                s_score[warp][lane + 32 * i] =
-                    a.routing == 1 ? 1.0f / (1.0f + expf(-lv[i])) : expf(lv[i] - m) / z;
-        __syncwarp();
-        for (int g = lane; g < G; g += 32) {
-            const float* s = &s_score[warp][g * gs];
-            float sc;
-            if (a.mode == 0) {
-                sc = s[0];
-                for (int i = 1; i < gs; ++i) sc = fmaxf(sc, s[i]);
-            } else {
-                int i1 = 0, i2 = -1;
-                for (int i = 1; i < gs; ++i)
-                    if (s[i] > s[i1]) i1 = i;
-                for (int i = 0; i < gs; ++i)
-                    if (i != i1 && (i2 < 0 || s[i] > s[i2])) i2 = i;
-                sc = s[i1] + s[i2];
-            }
-            s_gscore[warp][g] = sc;
-            s_sel[warp][g] = 0;                          // group taken flags
-        }
-        __syncwarp();
-        for (int r = 0; r < a.kg; ++r) {
-            float bv = -INFINITY;
-            int bi = -1;
-            for (int g = lane; g < G; g += 32) {
-                const float v = s_gscore[warp][g];
-                if (!s_sel[warp][g] && (bi < 0 || v > bv)) {   // ascending g: ties keep lower
-                    bv = v;
-                    bi = g;
-                }
-            }
-            argmax_reduce(bv, bi);
-            if (lane == 0) s_sel[warp][bi] = 1;
-            __syncwarp();
-        }
-        for (int e = lane; e < E; e += 32) s_elig[warp][e] = static_cast<unsigned char>(s_sel[warp][e / gs]);
-    } else {
-        for (int e = lane; e < E; e += 32) s_elig[warp][e] = 1;
-    }
-    __syncwarp();
-
-    // ---- top-k experts by logit among the eligible ones
-    uint32_t avail = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if ((okmask >> i & 1) && s_elig[warp][lane + 32 * i]) avail |= 1u << i;
-    for (int j = 0; j < a.K; ++j) {
-        float bv = -INFINITY;
-        int bi = -1;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if ((avail >> i & 1) && (bi < 0 || lv[i] > bv)) {   // ascending index: ties keep lower
-                bv = lv[i];
-                bi = lane + 32 * i;
-            }
-        }
-        argmax_reduce(bv, bi);
-        if (bi >= 0 && (bi & 31) == lane) avail &= ~(1u << (bi >> 5));
-        if (lane == 0) {
-            s_sel[warp][j] = bi;
-            s_score[warp][j] = bv;                       // the selected logit
-        }
-    }
-    __syncwarp();
-
-    // ---- weights (slot order, fp32)
-    if (lane == 0) {
-        const int K = a.K;
-        float* wv = s_gscore[warp];
-        float sum = 0.0f;
-        for (int j = 0; j < K; ++j) {
-            const float lj = s_score[warp][j];
-            const float v = a.routing == 1 ? 1.0f / (1.0f + expf(-lj)) : expf(lj - m) / z;
-            wv[j] = v;
-            sum += v;
-        }
-        const bool norm = a.routing == 1 || a.renorm;
-        for (int j = 0; j < K; ++j) {
-            const int e = s_sel[warp][j];
-            float v = norm ? wv[j] / sum : wv[j];
-            if (a.pes) v *= a.pes[e];
-            v *= a.rsf;
-            a.idx[static_cast<size_t>(t) * K + j] = e;
-            a.w[static_cast<size_t>(t) * K + j] = v;
-        }
-    }
+    route_token(a, t, lane, s_score[warp], s_gscore[warp], s_sel[warp], s_elig[warp], nullptr);
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
