@@ -81,12 +81,12 @@ __device__ __forceinline__ void decode_unit(int u, int nt, const int* tstart, in
     mb = local - nb * mt;
 }
 
-// acc[j] += P[j] * (sa * ws[j]) over 32 columns [c0, c0 + 32) already loaded into v; packed
+// acc[j] += P[j] * (sa * ws[j]) over 16 columns [c0, c0 + 16) already loaded into v; packed
 // fp32x2 multiply and FMA (each lane rounds as the scalar operations would).
-__device__ __forceinline__ void fma_chunk32(float2 (&acc)[kCols / 2], const uint32_t (&v)[32], const float* ws,
+__device__ __forceinline__ void fma_chunk16(float2 (&acc)[kCols / 2], const uint32_t (&v)[16], const float* ws,
                                             int c0, float2 sa2) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
+    for (int j = 0; j < 16; j += 4) {
         const float4 w4 = *reinterpret_cast<const float4*>(ws + c0 + j);
         const float2 s0 = __fmul2_rn(make_float2(w4.x, w4.y), sa2);
         const float2 s1 = __fmul2_rn(make_float2(w4.z, w4.w), sa2);
@@ -97,17 +97,23 @@ __device__ __forceinline__ void fma_chunk32(float2 (&acc)[kCols / 2], const uint
     }
 }
 
-// The promotion of one scale group over this thread's 64 columns: two rounds of one 32-column
-// TMEM load, its wait, then the multiply-adds.
+// The promotion of one scale group over this thread's 64 columns, software-pipelined in
+// 16-column chunks: the next chunk's TMEM load is in flight while the current one is multiplied in.
 __device__ __forceinline__ void promote_fp32(float2 (&acc)[kCols / 2], uint32_t taddr, const float* ws, float sa) {
     const float2 sa2 = make_float2(sa, sa);
-#pragma unroll
-    for (int c = 0; c < kCols; c += 32) {
-        uint32_t v[32];
-        MOE_TMEM_LD32(taddr + c, v);
-        MOE_TMEM_WAIT_LD(v);
-        fma_chunk32(acc, v, ws, c, sa2);
-    }
+    uint32_t a[16], b[16];
+    MOE_TMEM_LD16(taddr, a);
+    MOE_TMEM_WAIT_LD16(a);
+    MOE_TMEM_LD16(taddr + 16, b);
+    fma_chunk16(acc, a, ws, 0, sa2);
+    MOE_TMEM_WAIT_LD16(b);
+    MOE_TMEM_LD16(taddr + 32, a);
+    fma_chunk16(acc, b, ws, 16, sa2);
+    MOE_TMEM_WAIT_LD16(a);
+    MOE_TMEM_LD16(taddr + 48, b);
+    fma_chunk16(acc, a, ws, 32, sa2);
+    MOE_TMEM_WAIT_LD16(b);
+    fma_chunk16(acc, b, ws, 48, sa2);
 }
 
 }  // namespace
@@ -304,8 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float gt = acc[i], up = acc[32 + i];
-                        acc[i] = __fdiv_rn(gt, 1.0f + expf(-gt)) * up;
+                        acc[i] = silu(acc[i]) * acc[32 + i];
                     }
                 }
                 float amax = 0.0f;

@@ -16,6 +16,11 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
         if (globaltimer_ns() - t0 > kDrainLimitNs) break;
 }
 
+// silu(z) = z / (1 + e^-z), with the hardware exponential and a fast reciprocal division
+// (every GEMM kernel uses this same function, so their outputs agree bit for bit).  For z below
+// about -87 the divisor exceeds 2^126 and the quotient is 0, where the exact value is under 1e-36.
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
 // Add 32 bf16 bias values (16-byte aligned) to acc[0..31].
 __device__ __forceinline__ void add_bias32(float* acc, const __nv_bfloat16* bias) {
     const uint4* b4 = reinterpret_cast<const uint4*>(bias);

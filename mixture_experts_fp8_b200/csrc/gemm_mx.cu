@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
                 float amax = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    acc[i] = __fdiv_rn(acc[i], 1.0f + expf(-acc[i])) * acc[32 + i];
+                    acc[i] = silu(acc[i]) * acc[32 + i];
                     amax = fmaxf(amax, fabsf(acc[i]));
                 }
                 const int ex = mx_exponent(amax);

@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
                     }
                 }
 #pragma unroll
-                for (int t = 0; t < kNT; ++t) acc0[t] = __fdiv_rn(acc0[t], 1.0f + expf(-acc0[t])) * acc1[t];
+                for (int t = 0; t < kNT; ++t) acc0[t] = silu(acc0[t]) * acc1[t];
                 // per token, the maximum over the 128 act columns of this tile (four warps)
                 const int buf = tile & 1;
                 if (tile >= 2 && !mbar_wait(&amax_free[buf], ((tile >> 1) + 1) & 1, abort_flag, p.status)) {
