@@ -9,6 +9,13 @@
 // quantized SiLU products, then the down projection; "MATE Mega MoE", API: swiglu;
 // "MindIE-SD Fused MoE", parameter table: w13_bias / w2_bias.
 //
+// What bounds it: the scales vary with the row, the column and the 128-deep group, so every group
+// partial leaves the tensor core and is multiplied in, acc += P * (a_s * w_s): two fp32
+// operations per output element per group, as much FP32-pipe time as the MMAs themselves.  The
+// epilogue therefore keeps its per-group bookkeeping to a few instructions: per-lane barrier
+// arrivals (no divergent branches), no per-row predicates in the group loop, stage and phase
+// counters carried incrementally, 32-bit shared-memory addresses.
+//
 // Design (one persistent CTA per SM, 640 threads = five warpgroups):
 //   warp 0   TMA producer: per 128-deep K stage, a 128x128 A tile and a 256x128 B tile (both
 //            K-major, 128-byte swizzle), the 256 weight scales of the stage and the tile rows'
@@ -17,10 +24,11 @@
 //            scale group is accumulated alone into one of two 256-column fp32 TMEM buffers.
 //   warps 2-3 idle.  Warpgroup 0 gives registers back (setmaxnreg.dec to 32).
 //   warps 4-19 epilogue (setmaxnreg.inc to 112): warp w reads TMEM lanes 32*(w%4) .. +31 (tile
-//            rows) and one quarter of the columns; every group partial is multiplied by
-//            a_s * w_s and added into fp32 registers (the "promotion"), then the tile's epilogue
-//            runs from registers.  Four warps per lane quadrant keep the TMEM reads, which are
-//            the critical path of the promotion, in parallel.
+//            rows) and columns 32q .. +31 and 128 + 32q .. +31 of the tile, q = (w-4)/4; with
+//            w13's gate and up columns in 128-column blocks these are the gate and the up
+//            projections of the same 32 act columns.  Every group partial is multiplied by
+//            a_s * w_s and added into 64 fp32 registers (the "promotion"), then the tile's
+//            epilogue runs from registers.
 // Work unit = (expert, 256-column block, 128-row block), enumerated expert by expert, column
 // block, then row block; CTA c takes units c, c + grid, ...  Rows past an expert's end are
 // computed on whatever the tile holds and never stored.  Every wait is bounded.
@@ -36,14 +44,16 @@ constexpr int kStages = 4;
 constexpr int kThreads = 640;
 constexpr int kFirstEpiWarp = 4;
 constexpr int kEpiWarps = 16;
-constexpr int kCols = kTileN / 4;                  // columns per epilogue thread
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kCols = kTileN / 4;                  // columns per epilogue thread (32 per half)
+constexpr int kHalf = kTileN / 2;
 // Registers: 640 threads launch with 96 each (5 warps per SM sub-partition); warpgroup 0 keeps
 // 32, the four epilogue warpgroups take 112: 128 * 32 + 512 * 112 = 640 * 96.
 constexpr int kRegsLaunch = 96, kRegsLow = 32, kRegsHigh = 112;
 static_assert(128 * kRegsLow + 512 * kRegsHigh == kThreads * kRegsLaunch, "register split");
 constexpr uint32_t kABytes = kTileM * kTileK;      // 16 KB
 constexpr uint32_t kBBytes = kTileN * kTileK;      // 32 KB
-constexpr uint32_t kWsBytes = kTileN * 4;          // weight scales: fp32 or 4 x UE8M0 per column
+constexpr uint32_t kWsBytes = kTileN * 4;          // weight scales of the 256 columns
 constexpr uint32_t kSaWords = kTileM + 4;          // activation scales of the tile's rows (+ 16-byte alignment)
 constexpr uint32_t kSaBytes = kSaWords * 4;
 constexpr uint32_t kScaleSlot = 2048;              // per stage: [weight scales | activation scales]
@@ -53,14 +63,20 @@ struct L {
     static constexpr uint32_t a = 0;
     static constexpr uint32_t b = a + kStages * kABytes;
     static constexpr uint32_t sc = b + kStages * kBBytes;
-    static constexpr uint32_t bars = sc + kStages * kScaleSlot;
-    static constexpr uint32_t nbars = 2 * kStages + 7;   // full, empty, tfull[2], tempty[2], drain, amax[2]
-    static constexpr uint32_t misc = bars + nbars * 8;   // tmem holder, abort flag
+    // barriers: full[kStages], empty[kStages], tfull[2], tempty[2], drain, amax[2]
+    static constexpr uint32_t full = sc + kStages * kScaleSlot;
+    static constexpr uint32_t empty = full + 8 * kStages;
+    static constexpr uint32_t tfull = empty + 8 * kStages;
+    static constexpr uint32_t tempty = tfull + 16;
+    static constexpr uint32_t drain = tempty + 16;
+    static constexpr uint32_t amax_bar = drain + 8;
+    static constexpr uint32_t misc = amax_bar + 16;      // tmem holder, abort flag
     static constexpr uint32_t amax = misc + 16;          // float [2 buffers][4 quarters][128 rows]
     static constexpr uint32_t tstart = amax + 2 * 4 * 128 * 4;
     static constexpr uint32_t off = tstart + (MOE_MAX_EXPERTS + 1) * 4;
     static constexpr uint32_t end = off + (MOE_MAX_EXPERTS + 1) * 4;
 };
+static_assert(kWsBytes + kSaBytes <= kScaleSlot, "scale slot");
 constexpr uint32_t kSmemBytes = L::end + 1024;   // + slack to align the base to 1024 bytes
 static_assert(kSmemBytes <= 232448, "shared memory");
 
@@ -81,39 +97,20 @@ __device__ __forceinline__ void decode_unit(int u, int nt, const int* tstart, in
     mb = local - nb * mt;
 }
 
-// acc[j] += P[j] * (sa * ws[j]) over 16 columns [c0, c0 + 16) already loaded into v; packed
+// acc[a0 + j] += P[j] * (sa * ws[j]) for j < 16, with P in v and ws[] at shared address ws; packed
 // fp32x2 multiply and FMA (each lane rounds as the scalar operations would).
-__device__ __forceinline__ void fma_chunk16(float2 (&acc)[kCols / 2], const uint32_t (&v)[16], const float* ws,
-                                            int c0, float2 sa2) {
+__device__ __forceinline__ void fma_chunk16(float2 (&acc)[kCols / 2], const uint32_t (&v)[16], uint32_t ws,
+                                            int a0, float2 sa2) {
 #pragma unroll
     for (int j = 0; j < 16; j += 4) {
-        const float4 w4 = *reinterpret_cast<const float4*>(ws + c0 + j);
+        const float4 w4 = ld_shared_f32x4(ws + 4 * j);
         const float2 s0 = __fmul2_rn(make_float2(w4.x, w4.y), sa2);
         const float2 s1 = __fmul2_rn(make_float2(w4.z, w4.w), sa2);
-        acc[(c0 + j) / 2] = __ffma2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), s0,
-                                       acc[(c0 + j) / 2]);
-        acc[(c0 + j) / 2 + 1] = __ffma2_rn(make_float2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])), s1,
-                                           acc[(c0 + j) / 2 + 1]);
+        acc[(a0 + j) / 2] = __ffma2_rn(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), s0,
+                                       acc[(a0 + j) / 2]);
+        acc[(a0 + j) / 2 + 1] = __ffma2_rn(make_float2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3])), s1,
+                                           acc[(a0 + j) / 2 + 1]);
     }
-}
-
-// The promotion of one scale group over this thread's 64 columns, software-pipelined in
-// 16-column chunks: the next chunk's TMEM load is in flight while the current one is multiplied in.
-__device__ __forceinline__ void promote_fp32(float2 (&acc)[kCols / 2], uint32_t taddr, const float* ws, float sa) {
-    const float2 sa2 = make_float2(sa, sa);
-    uint32_t a[16], b[16];
-    MOE_TMEM_LD16(taddr, a);
-    MOE_TMEM_WAIT_LD16(a);
-    MOE_TMEM_LD16(taddr + 16, b);
-    fma_chunk16(acc, a, ws, 0, sa2);
-    MOE_TMEM_WAIT_LD16(b);
-    MOE_TMEM_LD16(taddr + 32, a);
-    fma_chunk16(acc, b, ws, 16, sa2);
-    MOE_TMEM_WAIT_LD16(a);
-    MOE_TMEM_LD16(taddr + 48, b);
-    fma_chunk16(acc, a, ws, 32, sa2);
-    MOE_TMEM_WAIT_LD16(b);
-    fma_chunk16(acc, b, ws, 48, sa2);
 }
 
 }  // namespace
@@ -127,12 +124,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::bars);
-    uint64_t* empty = full + kStages;
-    uint64_t* tfull = empty + kStages;
-    uint64_t* tempty = tfull + 2;
-    uint64_t* drain = tempty + 2;
-    uint64_t* amax_bar = drain + 1;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::full);
+    uint64_t* empty = reinterpret_cast<uint64_t*>(smem + L::empty);
+    uint64_t* tfull = reinterpret_cast<uint64_t*>(smem + L::tfull);
+    uint64_t* tempty = reinterpret_cast<uint64_t*>(smem + L::tempty);
+    uint64_t* drain = reinterpret_cast<uint64_t*>(smem + L::drain);
+    uint64_t* amax_bar = reinterpret_cast<uint64_t*>(smem + L::amax_bar);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc + 4);
     float* s_amax = reinterpret_cast<float*>(smem + L::amax);
@@ -143,12 +140,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + kEpiWarps);
+            mbar_init(&empty[s], 1 + kEpiThreads);   // the MMA commit + every epilogue thread
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kEpiWarps);
-            mbar_init(&amax_bar[b], kEpiWarps);
+            mbar_init(&tempty[b], kEpiThreads);
+            mbar_init(&amax_bar[b], kEpiThreads);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -168,9 +165,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int total_units = s_tstart[p.E] * nt;
-    const int KB = p.K / kTileK;                 // pipeline stages per unit
-    constexpr int GPS = 1;                       // scale groups per stage
-    constexpr int MPG = 4;                       // K=32 MMAs per scale group
+    const int KB = p.K / kTileK;                 // pipeline stages = scale groups per unit
+    constexpr int MPG = kTileK / 32;             // K=32 MMAs per scale group
 
     if (warp < kFirstEpiWarp) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
@@ -190,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint8_t* sa_src = static_cast<const uint8_t*>(p.a_scale) + static_cast<size_t>(row0 & ~3) * 4;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % kStages;
-                    if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, abort_flag, p.status)) {
+                    if (!mbar_wait<kProducerSleepNs>(&empty[s], ((it / kStages) & 1) ^ 1, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
@@ -210,34 +206,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (warp == 1 && lane == 0) {
             // -------------------------------------------------------------- MMA issuer
             const uint32_t idesc = f8_idesc(kTileM, kTileN);
-            uint32_t it = 0, kg = 0;
+            // descriptors of stage 0; a stage or a K step moves the start address field (bits
+            // 0..13, address / 16) by a fixed amount that never carries out of it
+            const uint64_t a_desc0 = sw128_kmajor_desc(smem_u32(smem + L::a));
+            const uint64_t b_desc0 = sw128_kmajor_desc(smem_u32(smem + L::b));
+            uint32_t s = 0, ph = 0, buf = 0, bph = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-                for (int kb = 0; kb < KB && ok; ++kb, ++it) {
-                    const int s = it % kStages;
-                    if (!mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status)) {
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait<kIssuerSleepNs>(&full[s], ph, abort_flag, p.status) ||
+                        !mbar_wait<kIssuerSleepNs>(&tempty[buf], bph ^ 1, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(smem + L::a + s * kABytes);
-                    const uint32_t b_addr = smem_u32(smem + L::b + s * kBBytes);
-                    for (int g = 0; g < GPS; ++g, ++kg) {
-                        const int b = kg & 1;
-                        if (!mbar_wait(&tempty[b], ((kg >> 1) & 1) ^ 1, abort_flag, p.status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t d = tmem_base + static_cast<uint32_t>(b * kTileN);
-                        for (int m = 0; m < MPG; ++m) {
-                            const uint32_t koff = static_cast<uint32_t>((g * MPG + m) * 32);
-                            mma_f8(d, sw128_kmajor_desc(a_addr + koff), sw128_kmajor_desc(b_addr + koff), idesc,
-                                   m > 0 ? 1u : 0u);
-                        }
-                        mma_commit(&tfull[b]);
+                    const uint64_t ad = a_desc0 + s * (kABytes >> 4), bd = b_desc0 + s * (kBBytes >> 4);
+                    const uint32_t d = tmem_base + buf * static_cast<uint32_t>(kTileN);
+#pragma unroll
+                    for (int m = 0; m < MPG; ++m) mma_f8(d, ad + 2 * m, bd + 2 * m, idesc, m > 0 ? 1u : 0u);
+                    mma_commit(&tfull[buf]);
+                    mma_commit(&empty[s]);
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1;
                     }
-                    if (ok) mma_commit(&empty[s]);
+                    buf ^= 1;
+                    bph ^= buf ^ 1;   // flips after both buffers were used
                 }
             }
             mma_commit(drain);          // all MMAs issued by this thread have finished
@@ -246,89 +240,107 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
         // ------------------------------------------------------------------ epilogue
-        const int ew = warp - kFirstEpiWarp;
         const int quad = warp & 3;                // TMEM lanes 32*quad .. 32*quad+31
-        const int qtr = ew >> 2;                  // columns qtr*64 .. qtr*64+63 of the tile
+        const int qtr = (warp - kFirstEpiWarp) >> 2;
         const int row_in_tile = quad * 32 + lane;
-        uint32_t it = 0, kg = 0, tile = 0;
+        // TMEM address of this thread's columns 32q.. (half 0) in buffer 0; its half-1 columns
+        // are 128 further.  Shared-memory addresses of its weight scales and of the activation-
+        // scale run in stage 0.
+        const uint32_t t_warp = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(32 * qtr);
+        const uint32_t ws0 = smem_u32(smem + L::sc) + static_cast<uint32_t>(32 * qtr * 4);
+        const uint32_t sa0 = smem_u32(smem + L::sc + kWsBytes) + static_cast<uint32_t>(row_in_tile * 4);
+        const uint32_t full0 = smem_u32(full), empty0 = smem_u32(empty);
+        const uint32_t tfull0 = smem_u32(tfull), tempty0 = smem_u32(tempty);
+        const uint32_t abort_at = smem_u32(smem + L::misc + 4);
+        uint32_t s = 0, ph = 0, buf = 0, bph = 0, tile = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++tile) {
-            int e, nb, mb;
-            decode_unit(u, nt, s_tstart, p.E, e, nb, mb);
-            const int row0 = s_off[e] + mb * kTileM;
-            const int cnt = min(kTileM, s_off[e + 1] - row0);
-            const bool warp_active = quad * 32 < cnt;
-            const bool row_ok = row_in_tile < cnt;
-            const int r = row0 + row_in_tile;
+            uint32_t sa_addr;
+            {
+                int e, nb, mb;
+                decode_unit(u, nt, s_tstart, p.E, e, nb, mb);
+                sa_addr = sa0 + static_cast<uint32_t>(((s_off[e] + mb * kTileM) & 3) * 4);
+            }
 
             float2 acc2[kCols / 2];
 #pragma unroll
             for (int i = 0; i < kCols / 2; ++i) acc2[i] = make_float2(0.0f, 0.0f);
             float* acc = reinterpret_cast<float*>(acc2);
 
-            for (int kb = 0; kb < KB && ok; ++kb, ++it) {
-                const int s = it % kStages;
-                // acquire the stage (its scales were written by the bulk copies)
-                if (!mbar_wait(&full[s], (it / kStages) & 1, abort_flag, p.status)) {
+            for (int kb = 0; kb < KB; ++kb) {
+                // the stage's scales (bulk copies), then the group partial in TMEM buffer buf
+                if (!mbar_wait_at(full0 + 8 * s, ph, abort_at, p.status) ||
+                    !mbar_wait_at(tfull0 + 8 * buf, bph, abort_at, p.status)) {
                     ok = false;
                     break;
                 }
-                const uint8_t* ws_stage = smem + L::sc + s * kScaleSlot + qtr * kCols * 4;
-                const uint32_t saw = reinterpret_cast<const uint32_t*>(smem + L::sc + s * kScaleSlot + kWsBytes)
-                    [(row0 & 3) + row_in_tile];
-                for (int g = 0; g < GPS; ++g, ++kg) {
-                    const int b = kg & 1;
-                    if (!mbar_wait(&tfull[b], (kg >> 1) & 1, abort_flag, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    if (warp_active) {
-                        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                               static_cast<uint32_t>(b * kTileN + qtr * kCols);
-                        promote_fp32(acc2, taddr, reinterpret_cast<const float*>(ws_stage), __uint_as_float(saw));
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[b]);
+                tc_fence_after();
+                const uint32_t so = s * kScaleSlot;
+                const float sa = ld_shared_f32(sa_addr + so);
+                const float2 sa2 = make_float2(sa, sa);
+                const uint32_t ws = ws0 + so;
+                const uint32_t taddr = t_warp + buf * static_cast<uint32_t>(kTileN);
+                // four 16-column chunks; each chunk's read overlaps the previous chunk's arithmetic
+                uint32_t va[16], vb[16];
+                MOE_TMEM_LD16(taddr, va);
+                MOE_TMEM_WAIT_LD16(va);
+                MOE_TMEM_LD16(taddr + 16, vb);
+                fma_chunk16(acc2, va, ws, 0, sa2);
+                MOE_TMEM_WAIT_LD16(vb);
+                MOE_TMEM_LD16(taddr + kHalf, va);
+                fma_chunk16(acc2, vb, ws + 64, 16, sa2);
+                MOE_TMEM_WAIT_LD16(va);
+                MOE_TMEM_LD16(taddr + kHalf + 16, vb);
+                fma_chunk16(acc2, va, ws + 4 * kHalf, 32, sa2);
+                MOE_TMEM_WAIT_LD16(vb);
+                // every read of buffer buf by this thread is complete: hand it back
+                tc_fence_before();
+                mbar_arrive_at(tempty0 + 8 * buf);
+                fma_chunk16(acc2, vb, ws + 4 * kHalf + 64, 48, sa2);
+                mbar_arrive_at(empty0 + 8 * s);      // done with the stage's scales
+                if (++s == kStages) {
+                    s = 0;
+                    ph ^= 1;
                 }
-                if (!ok) break;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
+                buf ^= 1;
+                bph ^= buf ^ 1;
             }
             if (!ok) break;
 
+            int e, nb, mb;
+            decode_unit(u, nt, s_tstart, p.E, e, nb, mb);
+            const int row0 = s_off[e] + mb * kTileM;
+            const int cnt = min(kTileM, s_off[e + 1] - row0);
+            const bool row_ok = row_in_tile < cnt;
+            const int r = row0 + row_in_tile;
             if (MODE == 0) {
-                // ---- SwiGLU + requantization.  This quarter holds acc[0:32] gate and acc[32:64] up
-                // of act columns c0 .. c0+31 (the transform's 32-column interleave).
+                // ---- SwiGLU + requantization: acc[0:32] gate (half 0) and acc[32:64] up (half 1)
+                // of act columns c0 .. c0+31.
                 const int I = p.N >> 1;
                 const int c0 = nb * 128 + qtr * 32;
-                if (warp_active) {
-                    if (p.bias) {
-                        add_bias32(acc, p.bias + static_cast<size_t>(e) * p.N + c0);
-                        add_bias32(acc + 32, p.bias + static_cast<size_t>(e) * p.N + I + c0);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        acc[i] = silu(acc[i]) * acc[32 + i];
-                    }
+                if (p.bias) {
+                    add_bias32(acc, p.bias + static_cast<size_t>(e) * p.N + c0);
+                    add_bias32(acc + 32, p.bias + static_cast<size_t>(e) * p.N + I + c0);
                 }
                 float amax = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(acc[i]));
+                for (int i = 0; i < 32; ++i) {
+                    acc[i] = silu(acc[i]) * acc[32 + i];
+                    amax = fmaxf(amax, fabsf(acc[i]));
+                }
                 // one 128-column group per row: combine the four quarters' maxima
-                const int buf = tile & 1;
-                s_amax[(buf * 4 + qtr) * 128 + row_in_tile] = amax;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&amax_bar[buf]);
-                if (!mbar_wait(&amax_bar[buf], (tile >> 1) & 1, abort_flag, p.status)) {
+                const int ab = tile & 1;
+                s_amax[(ab * 4 + qtr) * 128 + row_in_tile] = amax;
+                const uint32_t amax_at = smem_u32(&amax_bar[ab]);
+                mbar_arrive_at(amax_at);
+                if (!mbar_wait_at(amax_at, (tile >> 1) & 1, abort_at, p.status)) {
                     ok = false;
                     break;
                 }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) amax = fmaxf(amax, s_amax[(buf * 4 + q) * 128 + row_in_tile]);
+                for (int q = 0; q < 4; ++q) amax = fmaxf(amax, s_amax[(ab * 4 + q) * 128 + row_in_tile]);
                 const float sc = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-                if (warp_active && row_ok) {
+                if (row_ok) {
                     uint4* dst = reinterpret_cast<uint4*>(p.act_q + static_cast<size_t>(r) * I + c0);
 #pragma unroll
                     for (int w = 0; w < 2; ++w) {
@@ -346,17 +358,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (qtr == 0) static_cast<float*>(p.act_s)[static_cast<size_t>(nb) * p.a_pad + r] = sc;
                 }
             } else {
-                // ---- down projection: + bias, fp32 rows
-                const int c0 = nb * kTileN + qtr * kCols;
-                if (warp_active && row_ok && c0 < p.N) {
-                    if (p.bias) {
-                        add_bias32(acc, p.bias + static_cast<size_t>(e) * p.N + c0);
-                        add_bias32(acc + 32, p.bias + static_cast<size_t>(e) * p.N + c0 + 32);
-                    }
-                    float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.N + c0);
+                // ---- down projection: + bias, fp32 rows; acc[32h : 32h+32] are columns
+                // nb*256 + 128h + 32q .. +31
+                if (row_ok) {
 #pragma unroll
-                    for (int c = 0; c < kCols; c += 4)
-                        dst[c >> 2] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                    for (int h = 0; h < 2; ++h) {
+                        const int c0 = nb * kTileN + h * kHalf + qtr * 32;
+                        if (c0 < p.N) {
+                            float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.N + c0);
+                            const uint4* b4 =
+                                p.bias ? reinterpret_cast<const uint4*>(p.bias + static_cast<size_t>(e) * p.N + c0)
+                                       : nullptr;
+#pragma unroll
+                            for (int c = 0; c < 32; c += 8) {   // 8 columns: one bias load, two stores
+                                float* a = acc + 32 * h + c;
+                                if (b4) add_bias8(a, ld_nc_u4(b4 + (c >> 3)));
+                                dst[c >> 2] = make_float4(a[0], a[1], a[2], a[3]);
+                                dst[(c >> 2) + 1] = make_float4(a[4], a[5], a[6], a[7]);
+                            }
+                        }
+                    }
                 }
             }
         }
@@ -385,6 +406,9 @@ static cudaError_t launch_gemm_t(const GemmArgs& a, const CUtensorMap& tmA, cons
     if (e != cudaSuccess) return e;
     return launch_pdl(k_grouped_gemm<MODE>, dim3(num_sms), dim3(kThreads), kSmemBytes, s, tmA, tmB, a);
 }
+
+// Rows of the weight tensor-map box the wide kernel loads per stage (both modes).
+uint32_t gemm_weight_box(int) { return static_cast<uint32_t>(kTileN); }
 
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
                         cudaStream_t s) {

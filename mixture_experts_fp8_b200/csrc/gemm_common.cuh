@@ -12,28 +12,46 @@ constexpr unsigned long long kDrainLimitNs = 100000000ull;
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint32_t a = smem_u32(bar);
     const unsigned long long t0 = globaltimer_ns();
-    while (!mbar_try_wait(a, parity))
+    while (!mbar_try_wait(a, parity)) {
+        __nanosleep(128);
         if (globaltimer_ns() - t0 > kDrainLimitNs) break;
+    }
 }
+
+// Poll intervals of the single-thread roles, which mostly wait on the epilogue warps (the
+// producer for a free stage, the MMA issuer for a free accumulator): sleeping between polls keeps
+// them from taking issue slots on the schedulers they share with epilogue warps.
+constexpr uint32_t kProducerSleepNs = 256;
+constexpr uint32_t kIssuerSleepNs = 64;
 
 // silu(z) = z / (1 + e^-z), with the hardware exponential and a fast reciprocal division
 // (every GEMM kernel uses this same function, so their outputs agree bit for bit).  For z below
 // about -87 the divisor exceeds 2^126 and the quotient is 0, where the exact value is under 1e-36.
 __device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
+// Add 8 bf16 bias values (one 16-byte word) to acc[0..7].
+__device__ __forceinline__ void add_bias8(float* acc, uint4 w) {
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        acc[2 * q] += __uint_as_float(ww[q] << 16);
+        acc[2 * q + 1] += __uint_as_float(ww[q] & 0xFFFF0000u);
+    }
+}
+
+// A 16-byte read-only load kept in program order (volatile), so the compiler does not hoist all of
+// an epilogue's bias loads at once and run out of registers.
+__device__ __forceinline__ uint4 ld_nc_u4(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
 // Add 32 bf16 bias values (16-byte aligned) to acc[0..31].
 __device__ __forceinline__ void add_bias32(float* acc, const __nv_bfloat16* bias) {
     const uint4* b4 = reinterpret_cast<const uint4*>(bias);
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-        const uint4 w = __ldg(b4 + v);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            acc[8 * v + 2 * q] += __uint_as_float(ww[q] << 16);
-            acc[8 * v + 2 * q + 1] += __uint_as_float(ww[q] & 0xFFFF0000u);
-        }
-    }
+    for (int v = 0; v < 4; ++v) add_bias8(acc + 8 * v, ld_nc_u4(b4 + v));
 }
 
 }  // namespace moe

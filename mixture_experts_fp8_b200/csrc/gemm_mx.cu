@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
                                          (static_cast<size_t>(e) * nt + nb) * KB * kXSf;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % kXStages;
-                    if (!mbar_wait(&empty[s], ((it / kXStages) & 1) ^ 1, abort_flag, p.status)) {
+                    if (!mbar_wait<kProducerSleepNs>(&empty[s], ((it / kXStages) & 1) ^ 1, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
                 const uint32_t* src = static_cast<const uint32_t*>(p.a_scale) + static_cast<size_t>(kb) * p.a_pad + row0;
                 const uint4 w = make_uint4(__ldg(src + lane), __ldg(src + 32 + lane), __ldg(src + 64 + lane),
                                            __ldg(src + 96 + lane));
-                if (!mbar_wait(&empty[s], ((it / kXStages) & 1) ^ 1, abort_flag, p.status)) {
+                if (!mbar_wait<kProducerSleepNs>(&empty[s], ((it / kXStages) & 1) ^ 1, abort_flag, p.status)) {
                     ok = false;
                     break;
                 }
@@ -216,13 +216,13 @@ __global__ void __launch_bounds__(kXThreads, 1)
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++tile) {
                 const int b = tile & 1;
-                if (!mbar_wait(&tempty[b], ((tile >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+                if (!mbar_wait<kIssuerSleepNs>(&tempty[b], ((tile >> 1) & 1) ^ 1, abort_flag, p.status)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + static_cast<uint32_t>(b * kXN);
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % kXStages;
-                    if (!mbar_wait(&full[s], (it / kXStages) & 1, abort_flag, p.status) ||
-                        !mbar_wait(&sfready[s], (it / kXStages) & 1, abort_flag, p.status)) {
+                    if (!mbar_wait<kIssuerSleepNs>(&full[s], (it / kXStages) & 1, abort_flag, p.status) ||
+                        !mbar_wait<kIssuerSleepNs>(&sfready[s], (it / kXStages) & 1, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }

@@ -16,9 +16,9 @@
 // 4 KB per TMEM lane quadrant, and the kernel streams weights at HBM speed.
 //
 // Tile = (expert e, weight block wb, token block tb):
-//   mode 0: 128 gate rows and the 128 matching up rows of w13 (four 32-row chunks each, gathered
-//           by eight TMA loads from the interleaved transform) -> accumulators D0 (gate), D1 (up):
-//           lane j of both holds act column wb*128 + j, so SwiGLU stays in-thread.
+//   mode 0: 256 consecutive rows of the transformed w13, 128 gate rows and the 128 matching up
+//           rows -> accumulators D0 (gate), D1 (up): lane j of both holds act column wb*128 + j,
+//           so SwiGLU stays in-thread.
 //   mode 1: 256 consecutive rows of w2 -> D0 (rows 0..127), D1 (rows 128..255).
 // Threads: warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-7 epilogue (warp w reads
 // TMEM lanes 32*(w%4) .. +31), warps 2-3 idle.  Four TMEM accumulator pairs; every wait bounded.
@@ -157,23 +157,14 @@ __global__ void __launch_bounds__(kNThreads, 1)
                 const uint8_t* sa_src = static_cast<const uint8_t*>(p.a_scale) + static_cast<size_t>(row0 & ~3) * 4;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % kNStages;
-                    if (!mbar_wait(&empty[s], ((it / kNStages) & 1) ^ 1, abort_flag, p.status)) {
+                    if (!mbar_wait<kProducerSleepNs>(&empty[s], ((it / kNStages) & 1) ^ 1, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
                     uint8_t* st = smem + s * kStageBytes;
                     mbar_arrive_expect_tx(&full[s], kWBytes + kTBytes + ws_bytes + kNSaBytes);
-                    if (MODE == 0) {
-                        // gate rows (h = 0) and up rows (h = 1) of act columns wb*128 .. +127
-#pragma unroll
-                        for (int h = 0; h < 2; ++h)
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                tma_load_2d(st + h * 16384 + q * 4096, &tmW, kb * kTileK, wrow0 + q * 64 + h * 32,
-                                            &full[s]);
-                    } else {
-                        tma_load_2d(st, &tmW, kb * kTileK, wrow0, &full[s]);
-                    }
+                    // mode 0: the 128 gate rows, then the 128 up rows of act columns wb*128 .. +127
+                    tma_load_2d(st, &tmW, kb * kTileK, wrow0, &full[s]);
                     tma_load_2d(st + NL::t, &tmT, kb * kTileK, row0, &full[s]);
                     bulk_load(st + NL::ws, ws_src + static_cast<size_t>(kb) * p.N * 4, ws_bytes, &full[s]);
                     bulk_load(st + NL::sa, sa_src + static_cast<size_t>(kb) * p.a_pad * 4, kNSaBytes, &full[s]);
@@ -193,7 +184,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
                 for (int kb = 0; kb < KB && ok; ++kb, ++it) {
                     const int s = it % kNStages;
-                    if (!mbar_wait(&full[s], (it / kNStages) & 1, abort_flag, p.status)) {
+                    if (!mbar_wait<kIssuerSleepNs>(&full[s], (it / kNStages) & 1, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
@@ -202,7 +193,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
                     const uint32_t t_addr = w_addr + NL::t;
                     for (int g = 0; g < GPS; ++g, ++kg) {
                         const int b = kg % kNBuf;
-                        if (!mbar_wait(&tempty[b], ((kg / kNBuf) & 1) ^ 1, abort_flag, p.status)) {
+                        if (!mbar_wait<kIssuerSleepNs>(&tempty[b], ((kg / kNBuf) & 1) ^ 1, abort_flag, p.status)) {
                             ok = false;
                             break;
                         }
@@ -245,9 +236,9 @@ __global__ void __launch_bounds__(kNThreads, 1)
                 }
                 const uint8_t* st = smem + s * kStageBytes;
                 const uint32_t* wsw = reinterpret_cast<const uint32_t*>(st + NL::ws);
-                // this thread's two weight rows: gate/up of act column j (mode 0), or rows j, 128 + j
-                const uint32_t w0 = MODE == 0 ? wsw[(j >> 5) * 64 + (j & 31)] : wsw[j];
-                const uint32_t w1 = MODE == 0 ? wsw[(j >> 5) * 64 + 32 + (j & 31)] : wsw[128 + j];
+                // this thread's two weight rows j and 128 + j: gate and up of act column j in mode 0
+                const uint32_t w0 = wsw[j];
+                const uint32_t w1 = wsw[128 + j];
                 const uint32_t* saw = reinterpret_cast<const uint32_t*>(st + NL::sa) + (row0 & 3);
                 for (int g = 0; g < GPS; ++g, ++kg) {
                     const int b = kg % kNBuf;

@@ -34,6 +34,20 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Loads from a 32-bit shared-memory address (the data is written by the async proxy and made
+// visible by an mbarrier wait, so the loads must not be hoisted above it: volatile + memory).
+__device__ __forceinline__ float ld_shared_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 ld_shared_f32x4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a)
+                 : "memory");
+    return v;
+}
+
 // ------------------------------------------------------------------------------ warp helpers
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -111,18 +125,49 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up (returning false)
 // when *abort is set by another role, or after kWaitLimitNs, in which case it sets *abort and
-// records MOE_ERR_TIMEOUT.
+// records MOE_ERR_TIMEOUT.  kSleepNs > 0 makes a thread that has to wait sleep that long between
+// polls: for roles that wait on slower ones (a producer on its consumers), so that polling does
+// not take issue slots from the warps doing the work on the same scheduler.
+template <uint32_t kSleepNs = 0>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int32_t* status) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     unsigned long long t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
+        if (kSleepNs) __nanosleep(kSleepNs);
         if (mbar_try_wait(a, parity)) return true;
-        if ((i & 255u) == 0) {
+        if (kSleepNs || (i & 255u) == 0) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 *abort = 1;
+                set_status(status, MOE_ERR_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// The same two calls on 32-bit shared-memory addresses (the barrier's and the abort flag's), for
+// code that is short of registers: one 32-bit base stands in for several 64-bit pointers.
+__device__ __forceinline__ void mbar_arrive_at(uint32_t bar_addr) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_addr) : "memory");
+}
+
+template <uint32_t kSleepNs = 0>
+__device__ __forceinline__ bool mbar_wait_at(uint32_t bar_addr, uint32_t parity, uint32_t abort_addr,
+                                             int32_t* status) {
+    if (mbar_try_wait(bar_addr, parity)) return true;
+    unsigned long long t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (kSleepNs) __nanosleep(kSleepNs);
+        if (mbar_try_wait(bar_addr, parity)) return true;
+        if (kSleepNs || (i & 255u) == 0) {
+            uint32_t ab;
+            asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(ab) : "r"(abort_addr) : "memory");
+            if (ab) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(abort_addr), "r"(1u) : "memory");
                 set_status(status, MOE_ERR_TIMEOUT);
                 return false;
             }

@@ -82,6 +82,8 @@ cudaError_t launch_permute_small(const PermuteArgs& pa, bool clear_status, cudaS
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s);
+// Rows of the weight tensor-map box the wide kernel expects for each mode.
+uint32_t gemm_weight_box(int mode);
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         int num_sms, cudaStream_t s);
 cudaError_t launch_gemm_mx(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
@@ -93,22 +95,26 @@ constexpr int kNarrowRowsPerExpert = 32;
 int set_last_error(int code, const char* msg);
 cudaError_t launch_selftest_wait(int32_t* status, uint32_t timeout_us, cudaStream_t s);
 
-// Column permutation applied to w13 by the transform: within each 256-column block nb, four
-// 64-column quarters q = 0..3, each [gate nb*128 + 32q + 0:32 | up nb*128 + 32q + 0:32], so that
-// one GEMM epilogue thread holds matching gate and up columns.  Returns the transformed row index
-// of original column n (0 <= n < 2I).
-__host__ __device__ inline int w13_interleaved_row(int n, int I) {
+// Column permutation applied to w13 by the transform: the act columns are cut into blocks of
+// `blk` (128 for the fp32-scale recipe, 32 for MXFP8), and block j of gate columns is followed by
+// block j of up columns: transformed rows [2*blk*j, +blk) = gate j*blk .., [2*blk*j + blk, +blk) =
+// up I + j*blk ..  A GEMM epilogue thread then finds the gate and up columns of one act column in
+// the same place of the two halves of a 2*blk-column tile.  Returns the transformed row index of
+// original column n (0 <= n < 2I); I is a multiple of blk.
+__host__ __device__ inline int w13_interleaved_row(int n, int I, int blk) {
     const int is_up = n >= I;
     const int i = is_up ? n - I : n;
-    const int nb = i >> 7, within = i & 127;
-    return nb * 256 + (within >> 5) * 64 + is_up * 32 + (within & 31);
+    return (i / blk) * 2 * blk + is_up * blk + i % blk;
 }
 
 // Its inverse: the original column of transformed row r.
-__host__ __device__ inline int w13_original_col(int r, int I) {
-    const int nb = r >> 8, q = (r & 255) >> 6, is_up = (r & 63) >> 5, i = r & 31;
-    const int act = nb * 128 + q * 32 + i;
+__host__ __device__ inline int w13_original_col(int r, int I, int blk) {
+    const int j = r / (2 * blk), is_up = (r / blk) & 1, i = r % blk;
+    const int act = j * blk + i;
     return is_up ? I + act : act;
 }
+
+// The gate/up block of each recipe.
+__host__ __device__ inline int w13_block(int recipe) { return recipe == 1 ? 32 : 128; }
 
 }  // namespace moe

@@ -323,8 +323,8 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     const bool narrow = !mx && A <= moe::kNarrowRowsPerExpert * E;
     CUtensorMap tm_x, tm_w13, tm_act, tm_w2;
     const uint32_t tok_box = narrow ? 16 : moe::kTileM;
-    const uint32_t w13_box = mx ? 128 : narrow ? 32 : moe::kTileN;
-    const uint32_t w2_box = mx ? 128 : moe::kTileN;
+    const uint32_t w13_box = mx ? 128 : narrow ? moe::kTileN : moe::gemm_weight_box(0);
+    const uint32_t w2_box = mx ? 128 : narrow ? moe::kTileN : moe::gemm_weight_box(1);
     if ((rc = make_kmajor_map(&tm_x, at(L.xq), A, H, tok_box))) return rc;
     if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(E) * 2 * I, H, w13_box))) return rc;
     if ((rc = make_kmajor_map(&tm_act, at(L.act_q), A, I, tok_box))) return rc;

@@ -104,14 +104,15 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
 }
 
 // ------------------------------------------------------------------------------------------
-// Weight transform (offline): E4M3 codes [E, K, N] -> K-major [E, N', K], with w13's columns
-// interleaved (moe::w13_interleaved_row), and the block scales re-laid to match:
+// Weight transform (offline): E4M3 codes [E, K, N] -> K-major [E, N', K], with w13's gate and up
+// columns interleaved in blocks (moe::w13_interleaved_row, moe::w13_block), and the block scales
+// re-laid to match:
 //   recipe 0: fp32 [E, K/128, N] -> [E, K/128, N'] (columns permuted like the codes)
 //   recipe 1: UE8M0 [E, K/32, N] -> 512-byte scale-factor atoms [E, N/128, K/128] for the
 //             block-scaled tensor core (see gemm_mx.cu)
 // ("MATE Mega MoE", transform_weights_for_mega_moe; "DeepGEMM PR #371", 4-packed UE8M0.)
 __global__ void __launch_bounds__(256) k_transpose_codes(const uint8_t* src, uint8_t* dst, int K,
-                                                        int N, int interleave_I) {
+                                                        int N, int interleave_I, int blk) {
     __shared__ uint8_t tile[64][65];
     const int e = blockIdx.z;
     const int k0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(256) k_transpose_codes(const uint8_t* src, uin
         const int nn = i / 64, kk = i % 64;
         const int n = n0 + nn, k = k0 + kk;
         if (n < N && k < K) {
-            const int row = interleave_I ? w13_interleaved_row(n, interleave_I) : n;
+            const int row = interleave_I ? w13_interleaved_row(n, interleave_I, blk) : n;
             d[static_cast<size_t>(row) * K + k] = tile[kk][nn];
         }
     }
@@ -134,6 +135,7 @@ __global__ void __launch_bounds__(256) k_transpose_codes(const uint8_t* src, uin
 
 __global__ void k_transform_scales(const void* src, void* dst, int E, int K, int N, int recipe,
                                    int interleave_I) {
+    const int blk = w13_block(recipe);
     if (recipe == 0) {
         // fp32 [E, K/128, N] -> [E, K/128, N'] (columns permuted like the codes)
         const size_t total = static_cast<size_t>(E) * (K / 128) * N;
@@ -141,7 +143,7 @@ __global__ void k_transform_scales(const void* src, void* dst, int E, int K, int
              i += static_cast<size_t>(gridDim.x) * blockDim.x) {
             const int n = static_cast<int>(i % N);
             const size_t ek = i / N;                    // e * (K/128) + kb
-            const int row = interleave_I ? w13_interleaved_row(n, interleave_I) : n;
+            const int row = interleave_I ? w13_interleaved_row(n, interleave_I, blk) : n;
             static_cast<float*>(dst)[ek * N + row] = static_cast<const float*>(src)[ek * N + n];
         }
         return;
@@ -163,15 +165,16 @@ __global__ void k_transform_scales(const void* src, void* dst, int E, int K, int
         const size_t e = enb / NB;
         const int i = byte >> 4, c = (byte >> 2) & 3, k = byte & 3;
         const int row = nb * 128 + 32 * c + i;
-        const int col = interleave_I ? w13_original_col(row, interleave_I) : row;
+        const int col = interleave_I ? w13_original_col(row, interleave_I, blk) : row;
         d[idx] = s[(e * (K / 32) + kb * 4 + k) * N + col];
     }
 }
 
 cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s) {
     const int H = a.H, I = a.I, E = a.E;
-    k_transpose_codes<<<dim3((2 * I + 63) / 64, (H + 63) / 64, E), 256, 0, s>>>(a.w13, a.w13_t, H, 2 * I, I);
-    k_transpose_codes<<<dim3((H + 63) / 64, (I + 63) / 64, E), 256, 0, s>>>(a.w2, a.w2_t, I, H, 0);
+    k_transpose_codes<<<dim3((2 * I + 63) / 64, (H + 63) / 64, E), 256, 0, s>>>(a.w13, a.w13_t, H, 2 * I, I,
+                                                                                 w13_block(a.recipe));
+    k_transpose_codes<<<dim3((H + 63) / 64, (I + 63) / 64, E), 256, 0, s>>>(a.w2, a.w2_t, I, H, 0, 1);
     k_transform_scales<<<1024, 256, 0, s>>>(a.w13s, a.w13s_t, E, H, 2 * I, a.recipe, I);
     k_transform_scales<<<1024, 256, 0, s>>>(a.w2s, a.w2s_t, E, I, H, a.recipe, 0);
     return cudaGetLastError();

@@ -85,11 +85,15 @@ def test_forward_rejects_bad_pointers_before_any_cuda_call():
 
 
 def test_interleave_is_a_permutation():
-    # mirror of the transform's column order, checked for bijectivity
-    I = 384
-    def row(n):
-        up = n >= I
-        i = n - I if up else n
-        return (i >> 7) * 256 + ((i & 127) >> 5) * 64 + up * 32 + (i & 31)
-    rows = sorted(row(n) for n in range(2 * I))
-    assert rows == list(range(2 * I))
+    # mirror of the transform's gate/up column order (blocks of 128 for the fp32-scale recipe,
+    # 32 for MXFP8), checked for bijectivity and for gate/up pairing at the same offset
+    for blk in (128, 32):
+        I = 384
+        def row(n):
+            up = n >= I
+            i = n - I if up else n
+            return (i // blk) * 2 * blk + up * blk + i % blk
+        rows = [row(n) for n in range(2 * I)]
+        assert sorted(rows) == list(range(2 * I))
+        for i in range(I):
+            assert rows[I + i] - rows[i] == blk
