@@ -12,9 +12,9 @@
 // What bounds it: the scales vary with the row, the column and the 128-deep group, so every group
 // partial leaves the tensor core and is multiplied in, acc += P * (a_s * w_s): two fp32
 // operations per output element per group, as much FP32-pipe time as the MMAs themselves.  The
-// epilogue therefore keeps its per-group bookkeeping to a few instructions: per-lane barrier
-// arrivals (no divergent branches), no per-row predicates in the group loop, stage and phase
-// counters carried incrementally, 32-bit shared-memory addresses.
+// epilogue therefore keeps its per-group bookkeeping to a few instructions: one predicated barrier
+// arrival per warp (no divergent branches), no per-row predicates in the group loop, stage and
+// phase counters carried incrementally, 32-bit shared-memory addresses.
 //
 // Design (one persistent CTA per SM, 640 threads = five warpgroups):
 //   warp 0   TMA producer: per 128-deep K stage, a 128x128 A tile and a 256x128 B tile (both
@@ -44,7 +44,6 @@ constexpr int kStages = 4;
 constexpr int kThreads = 640;
 constexpr int kFirstEpiWarp = 4;
 constexpr int kEpiWarps = 16;
-constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kCols = kTileN / 4;                  // columns per epilogue thread (32 per half)
 constexpr int kHalf = kTileN / 2;
 // Registers: 640 threads launch with 96 each (5 warps per SM sub-partition); warpgroup 0 keeps
@@ -140,12 +139,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1 + kEpiThreads);   // the MMA commit + every epilogue thread
+            mbar_init(&empty[s], 1 + kEpiWarps);   // the MMA commit + one arrival per epilogue warp
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], kEpiThreads);
-            mbar_init(&amax_bar[b], kEpiThreads);
+            mbar_init(&tempty[b], kEpiWarps);
+            mbar_init(&amax_bar[b], kEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -293,11 +292,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 MOE_TMEM_LD16(taddr + kHalf + 16, vb);
                 fma_chunk16(acc2, va, ws + 4 * kHalf, 32, sa2);
                 MOE_TMEM_WAIT_LD16(vb);
-                // every read of buffer buf by this thread is complete: hand it back
+                // every read of buffer buf by this warp is complete: hand it back
                 tc_fence_before();
-                mbar_arrive_at(tempty0 + 8 * buf);
+                mbar_arrive_lane0(tempty0 + 8 * buf, lane);
                 fma_chunk16(acc2, vb, ws + 4 * kHalf + 64, 48, sa2);
-                mbar_arrive_at(empty0 + 8 * s);      // done with the stage's scales
+                mbar_arrive_lane0(empty0 + 8 * s, lane);   // done with the stage's scales
                 if (++s == kStages) {
                     s = 0;
                     ph ^= 1;
@@ -332,7 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int ab = tile & 1;
                 s_amax[(ab * 4 + qtr) * 128 + row_in_tile] = amax;
                 const uint32_t amax_at = smem_u32(&amax_bar[ab]);
-                mbar_arrive_at(amax_at);
+                __syncwarp();                          // every lane's s_amax store before the arrival
+                mbar_arrive_lane0(amax_at, lane);
                 if (!mbar_wait_at(amax_at, (tile >> 1) & 1, abort_at, p.status)) {
                     ok = false;
                     break;

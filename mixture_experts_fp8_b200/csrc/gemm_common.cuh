@@ -22,7 +22,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 // producer for a free stage, the MMA issuer for a free accumulator): sleeping between polls keeps
 // them from taking issue slots on the schedulers they share with epilogue warps.
 constexpr uint32_t kProducerSleepNs = 256;
-constexpr uint32_t kIssuerSleepNs = 64;
+constexpr uint32_t kIssuerSleepNs = 0;
 
 // silu(z) = z / (1 + e^-z), with the hardware exponential and a fast reciprocal division
 // (every GEMM kernel uses this same function, so their outputs agree bit for bit).  For z below

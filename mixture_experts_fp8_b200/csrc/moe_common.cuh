@@ -154,6 +154,17 @@ __device__ __forceinline__ void mbar_arrive_at(uint32_t bar_addr) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_addr) : "memory");
 }
 
+// One arrival from lane 0 of the warp, predicated inside the asm (no divergent branch).  For use
+// after warp-collective operations (tcgen05.wait::ld, or loads whose values the whole warp has
+// consumed), which every lane has completed when lane 0 gets here.
+__device__ __forceinline__ void mbar_arrive_lane0(uint32_t bar_addr, int lane) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.s32 p, %1, 0;\n\t@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(
+            bar_addr),
+        "r"(lane)
+        : "memory");
+}
+
 template <uint32_t kSleepNs = 0>
 __device__ __forceinline__ bool mbar_wait_at(uint32_t bar_addr, uint32_t parity, uint32_t abort_addr,
                                              int32_t* status) {
