@@ -36,7 +36,12 @@ import synth  # noqa: E402
 METRIC = "MoE-layer tokens/s & FP8 TFLOPS (% of tensor/HBM roofline), 1×B200"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
-KERNELS_PER_STEP = 8         # route, hist, scan, scatter, quant, gemm1, gemm2, combine
+SMALL_ROWS = 2048             # the library permutes up to this many routed rows in one launch
+
+
+def kernels_per_step(A: int) -> int:
+    # route, permute (one kernel, or histogram + scan + scatter), quantize, gemm1, gemm2, combine
+    return 6 if A <= SMALL_ROWS else 8
 
 
 def peaks():
@@ -348,8 +353,11 @@ def main():
                     "frac": g1_tflops / fp8_peak}
         else:
             roof = {"bound": "hbm", "achieved": g1_gbs, "peak": hbm, "unit": "GB/s", "frac": g1_gbs / hbm}
-        narrow = A <= 32 * shape.num_experts     # the library's rule for the swap-AB kernels
-        roof.update({"kernel": ("k_grouped_gemm_narrow" if narrow else "k_grouped_gemm") + "<gate+up>",
+        # the library's kernel choice: MXFP8 -> block-scaled kernel; fp32 scales -> swap-AB narrow
+        # kernel at <= 32 routed rows per expert, else the wide kernel
+        kname = ("k_grouped_gemm_mx" if shape.recipe == 1 else
+                 "k_grouped_gemm_narrow" if A <= 32 * shape.num_experts else "k_grouped_gemm")
+        roof.update({"kernel": kname + "<gate+up>",
                      "traffic": traffic_for("gemm1", shape.name),
                      "peak_source": f"{pk_kind} ({'sustained bf16 x2 for fp8' if compute_bound else 'copy'})",
                      "algorithmic_bytes_per_launch": g1_bytes, "ms_per_launch": g1_ms})
@@ -369,7 +377,7 @@ def main():
             "stages_ms": {k: v / max(calls, 1) for k, v in stage_ms.items()},
             "ms_per_step_with_stage_events": ms_profiled / args.steps,
             "gemm2": {"ms": g2_ms, "GB/s": gemm2_bytes(shape, active) / (g2_ms / 1e3) / 1e9},
-            "clocks": clocks, "gpu_launches": KERNELS_PER_STEP * args.steps, "status": status,
+            "clocks": clocks, "gpu_launches": kernels_per_step(A) * args.steps, "status": status,
             "e2e": {"value": world * shape.num_tokens * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_h.numel() * 2 + l_h.numel() * 4,
                     "d2h_bytes_per_step": y_h.numel() * 2},
