@@ -8,7 +8,19 @@
 
 namespace moe {
 
-constexpr int kPermuteChunk = 256;    // routed rows per histogram / scatter chunk
+constexpr int kPermuteChunk = 256;    // granularity of the histogram / scatter chunks (routed rows)
+constexpr int kMaxPermuteChunks = 64; // the per-expert scan over chunks stays this short
+// Rows per chunk: a multiple of kPermuteChunk, large enough that there are at most
+// kMaxPermuteChunks chunks.
+inline int permute_chunk_rows(long long A) {
+    const long long units = (A + kPermuteChunk - 1) / kPermuteChunk;
+    const long long per = (units + kMaxPermuteChunks - 1) / kMaxPermuteChunks;
+    return kPermuteChunk * static_cast<int>(per > 0 ? per : 1);
+}
+inline int permute_chunks(long long A) {
+    const int rows = permute_chunk_rows(A);
+    return static_cast<int>((A + rows - 1) / rows);
+}
 constexpr int kSmallRows = 2048;      // batches up to this many routed rows are permuted by one block
 constexpr int kTileM = 128;           // GEMM rows per tile
 constexpr int kTileN = 256;           // GEMM output columns per tile
@@ -34,7 +46,7 @@ struct PermuteArgs {
     int32_t* row_of;            // [A]
     int32_t* expert_counts;     // [E] or null (caller's copy)
     int32_t* status;
-    int A, E, chunks;
+    int A, E, chunks, chunk;    // chunk = routed rows per chunk
 };
 
 struct QuantArgs {

@@ -89,7 +89,7 @@ size_t scale_rows_of(size_t A) { return align_up(A + moe::kTileM + 4, 4); }
 void layout_of(const moe_config_t* c, moe_workspace_layout_t* L) {
     const size_t T = c->num_tokens, K = c->top_k, E = c->num_experts, H = c->hidden, I = c->inter;
     const size_t A = T * K, SR = scale_rows_of(A);
-    const size_t chunks = (A + moe::kPermuteChunk - 1) / moe::kPermuteChunk;
+    const size_t chunks = moe::permute_chunks(static_cast<long long>(A));
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
@@ -342,7 +342,7 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     moe::PermuteArgs pa{idx, static_cast<int32_t*>(at(L.hist)), static_cast<int32_t*>(at(L.counts)),
                         static_cast<int32_t*>(at(L.offsets)), static_cast<int32_t*>(at(L.tile_start)),
                         static_cast<int32_t*>(at(L.row_src)), static_cast<int32_t*>(at(L.row_of)), expert_counts,
-                        status, A, E, (A + moe::kPermuteChunk - 1) / moe::kPermuteChunk};
+                        status, A, E, moe::permute_chunks(A), moe::permute_chunk_rows(A)};
     MOE_CUDA_TRY(mark(0));
     // The first kernel of the forward clears the status word: the router when it runs, else the
     // small-batch permutation; a memset otherwise.

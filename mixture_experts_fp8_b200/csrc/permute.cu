@@ -4,11 +4,13 @@
 // expert's tokens; combine restores token order.  Routed row a = t*k + j; inside an expert,
 // rows keep ascending a (hence ascending token).  Three launches, no global atomics, so the
 // result is the same bits on every run:
-//   1. k_hist     per-chunk expert histograms (chunk = kPermuteChunk routed rows)
+//   1. k_hist     per-chunk expert histograms (a chunk is a multiple of kPermuteChunk routed
+//                 rows, sized so that there are at most kMaxPermuteChunks chunks)
 //   2. k_scan     per-expert exclusive bases across chunks, counts, offsets = exclusive scan,
 //                 and the first 128-row GEMM tile of every expert
 //   3. k_scatter  one warp per chunk walks its rows in order; rows with the same expert inside
 //                 a 32-row batch are ranked with a warp match.
+// Bounding the chunk count keeps k_scan's serial walk over the chunks short for large batches.
 #include "moe_common.cuh"
 #include "moe_kernels.h"
 
@@ -19,8 +21,8 @@ __global__ void __launch_bounds__(256) k_hist(PermuteArgs a) {
     pdl_wait_then_release();
     for (int e = threadIdx.x; e < a.E; e += blockDim.x) cnt[e] = 0;
     __syncthreads();
-    const int begin = blockIdx.x * kPermuteChunk;
-    const int end = min(a.A, begin + kPermuteChunk);
+    const int begin = blockIdx.x * a.chunk;
+    const int end = min(a.A, begin + a.chunk);
     for (int r = begin + threadIdx.x; r < end; r += blockDim.x) {
         const int e = a.idx[r];
         if (e >= 0 && e < a.E) atomicAdd(&cnt[e], 1);
@@ -62,14 +64,17 @@ __global__ void __launch_bounds__(256) k_scan(PermuteArgs a) {
     __shared__ int tmp[16];
     pdl_wait_then_release();
     const int e = threadIdx.x;
+    // all of this expert's chunk counts are loaded at once (at most kMaxPermuteChunks), then
+    // replaced by their exclusive prefix
+    int v[kMaxPermuteChunks];
+#pragma unroll
+    for (int c = 0; c < kMaxPermuteChunks; ++c)
+        v[c] = (e < a.E && c < a.chunks) ? a.hist[static_cast<size_t>(c) * a.E + e] : 0;
     int run = 0;
-    if (e < a.E) {
-        for (int c = 0; c < a.chunks; ++c) {
-            int32_t* h = a.hist + static_cast<size_t>(c) * a.E + e;
-            const int v = *h;
-            *h = run;
-            run += v;
-        }
+#pragma unroll
+    for (int c = 0; c < kMaxPermuteChunks; ++c) {
+        if (e < a.E && c < a.chunks) a.hist[static_cast<size_t>(c) * a.E + e] = run;
+        run += v[c];
     }
     const int cnt = e < a.E ? run : 0;
     const int off = block_exclusive_scan_256(cnt, tmp);
@@ -92,35 +97,37 @@ __global__ void __launch_bounds__(32) k_scatter(PermuteArgs a) {
     constexpr int kBatches = kPermuteChunk / 32;
     pdl_wait_then_release();
     const int lane = threadIdx.x;
-    const int begin = blockIdx.x * kPermuteChunk;
-    const int end = min(a.A, begin + kPermuteChunk);
-    int ids[kBatches];                                  // all of the chunk's ids, loaded at once
-#pragma unroll
-    for (int b = 0; b < kBatches; ++b) {
-        const int r = begin + 32 * b + lane;
-        ids[b] = r < end ? a.idx[r] : -1;
-    }
+    const int begin = blockIdx.x * a.chunk;
+    const int end = min(a.A, begin + a.chunk);
     for (int e = lane; e < a.E; e += 32)
         base[e] = a.offsets[e] + a.hist[static_cast<size_t>(blockIdx.x) * a.E + e];
     __syncwarp();
+    for (int p0 = begin; p0 < end; p0 += kPermuteChunk) {
+        int ids[kBatches];                              // the next 256 ids, loaded at once
 #pragma unroll
-    for (int b = 0; b < kBatches; ++b) {
-        const int r = begin + 32 * b + lane;
-        const bool valid = r < end;
-        int e = ids[b];
-        if (e >= a.E) e = -1;                           // reported by k_hist
-        const uint32_t active = __ballot_sync(0xffffffffu, valid && e >= 0);
-        const uint32_t peers = __match_any_sync(0xffffffffu, e);
-        const uint32_t mine = peers & active;
-        const int rank = __popc(mine & ((1u << lane) - 1u));
-        int dst = 0;
-        if (valid && e >= 0) dst = base[e] + rank;
-        __syncwarp();
-        if (valid && e >= 0 && rank == 0) base[e] += __popc(mine);
-        __syncwarp();
-        if (valid && e >= 0) {
-            a.row_src[dst] = r;
-            a.row_of[r] = dst;
+        for (int b = 0; b < kBatches; ++b) {
+            const int r = p0 + 32 * b + lane;
+            ids[b] = r < end ? a.idx[r] : -1;
+        }
+#pragma unroll
+        for (int b = 0; b < kBatches; ++b) {
+            const int r = p0 + 32 * b + lane;
+            const bool valid = r < end;
+            int e = ids[b];
+            if (e >= a.E) e = -1;                       // reported by k_hist
+            const uint32_t active = __ballot_sync(0xffffffffu, valid && e >= 0);
+            const uint32_t peers = __match_any_sync(0xffffffffu, e);
+            const uint32_t mine = peers & active;
+            const int rank = __popc(mine & ((1u << lane) - 1u));
+            int dst = 0;
+            if (valid && e >= 0) dst = base[e] + rank;
+            __syncwarp();
+            if (valid && e >= 0 && rank == 0) base[e] += __popc(mine);
+            __syncwarp();
+            if (valid && e >= 0) {
+                a.row_src[dst] = r;
+                a.row_of[r] = dst;
+            }
         }
     }
 }

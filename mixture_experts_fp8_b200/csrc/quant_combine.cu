@@ -44,18 +44,28 @@ __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
         q = e4m3x4(v0 * inv, v1 * inv, v2 * inv, v3 * inv);
         e8 = static_cast<uint8_t>(e + 127);
     }
+    // the token's destination rows: lane j holds row_of[t, j] (slots past 32 are read in the loop)
     const int A = a.T * a.K;
+    const int32_t* rows = a.row_of + static_cast<size_t>(t) * a.K;
+    const int r_lane = lane < a.K ? __ldg(rows + lane) : -1;
+    const bool lane_row_ok = r_lane >= 0 && r_lane < A;
+    if (lane < a.K && !lane_row_ok) set_status(a.status, MOE_ERR_BOUNDS);
     for (int j = 0; j < a.K; ++j) {
-        const int r = a.row_of[static_cast<size_t>(t) * a.K + j];
+        const int r = j < 32 ? __shfl_sync(0xffffffffu, r_lane, j) : __ldg(rows + j);
         if (r < 0 || r >= A) {
-            if (lane == 0) set_status(a.status, MOE_ERR_BOUNDS);
+            if (j >= 32 && lane == 0) set_status(a.status, MOE_ERR_BOUNDS);
             continue;
         }
         *reinterpret_cast<uint32_t*>(a.xq + static_cast<size_t>(r) * a.H + cb * 128 + 4 * lane) = q;
-        if (a.recipe == 0) {
-            if (lane == 0) static_cast<float*>(a.xs)[static_cast<size_t>(cb) * a.a_pad + r] = s32;
-        } else if ((lane & 7) == 0) {
+        if (a.recipe == 1 && (lane & 7) == 0)
             static_cast<uint8_t*>(a.xs)[(static_cast<size_t>(cb) * a.a_pad + r) * 4 + (lane >> 3)] = e8;
+    }
+    // fp32 scales: lane j stores the scale of the token's j-th row (one instruction for up to 32)
+    if (a.recipe == 0) {
+        if (lane < a.K && lane_row_ok) static_cast<float*>(a.xs)[static_cast<size_t>(cb) * a.a_pad + r_lane] = s32;
+        for (int j = 32 + lane; j < a.K; j += 32) {
+            const int r = __ldg(rows + j);
+            if (r >= 0 && r < A) static_cast<float*>(a.xs)[static_cast<size_t>(cb) * a.a_pad + r] = s32;
         }
     }
 }
