@@ -224,6 +224,17 @@ int moe_read_status(const void *workspace, int32_t *status, void *stream);
  * the device int32 *status and returns.  The context stays usable. */
 int moe_selftest_bounded_wait(int32_t *status, uint32_t timeout_us, void *stream);
 
+/* Fault injection for failure-detection tests (no counterpart on the pages).  Only the debug
+ * library, libmoefp8_debug.so (built with MOE_FAULT_INJECTION), acts on it; the release library
+ * returns MOE_ERR_UNSUPPORTED.  MOE_FAULT_SKIP_STAGE arms one fault for the next moe_forward on
+ * this host thread: the gate+up GEMM's producer in CTA 0 skips its first K stage (no copies, no
+ * arrival), so the MMA role's bounded wait runs out (about 2 s), every role of that CTA leaves
+ * cleanly and the status word reads MOE_ERR_TIMEOUT.  Nothing faults or hangs; the context stays
+ * usable.  MOE_FAULT_NONE disarms it. */
+#define MOE_FAULT_NONE 0
+#define MOE_FAULT_SKIP_STAGE 1
+int moe_debug_inject_fault(int fault);
+
 #ifdef __cplusplus
 }
 #endif

@@ -35,7 +35,10 @@ EXPORTED = (
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_forward", "moe_forward_profiled",
     "moe_profile_create", "moe_profile_destroy", "moe_profile_read", "moe_profile_reset",
     "moe_read_status", "moe_selftest_bounded_wait", "moe_forward_static_workspace",
+    "moe_debug_inject_fault",
 )
+MOE_FAULT_NONE = 0
+MOE_FAULT_SKIP_STAGE = 1
 
 
 class MoeError(RuntimeError):
@@ -125,6 +128,7 @@ def _load():
             "moe_read_status": [P, P, P],
             "moe_selftest_bounded_wait": [P, ctypes.c_uint32, P],
             "moe_forward_static_workspace": [CP] + [P] * 13 + [P],
+            "moe_debug_inject_fault": [I],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -261,6 +265,12 @@ def read_status(workspace, stream=None) -> int:
 
 def selftest_bounded_wait(status_tensor, timeout_us: int, stream=None) -> None:
     _check(_load().moe_selftest_bounded_wait(_ptr(status_tensor), int(timeout_us), _stream(stream)))
+
+
+def debug_inject_fault(fault: int) -> None:
+    """Arm a fault for the next forward on this thread (the debug library only; the release
+    library raises MoeError with MOE_ERR_UNSUPPORTED)."""
+    _check(_load().moe_debug_inject_fault(int(fault)))
 
 
 class Profile:

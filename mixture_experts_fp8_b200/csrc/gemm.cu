@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (fault_skip_stage(p.fault, it)) continue;   // debug builds: an injected fault
                     mbar_arrive_expect_tx(&full[s], kABytes + kBBytes + ws_bytes + kSaBytes);
                     tma_load_2d(smem + L::a + s * kABytes, &tmA, kb * kTileK, row0, &full[s]);
                     tma_load_2d(smem + L::b + s * kBBytes, &tmB, kb * kTileK, brow0, &full[s]);

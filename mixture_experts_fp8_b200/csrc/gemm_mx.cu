@@ -173,6 +173,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (fault_skip_stage(p.fault, it)) continue;   // debug builds: an injected fault
                     uint8_t* st = smem + s * kXStage;
                     mbar_arrive_expect_tx(&full[s], kXA + kXB + kXSf);
                     tma_load_2d(st, &tmA, kb * kTileK, row0, &full[s]);

@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(kNThreads, 1)
                         ok = false;
                         break;
                     }
+                    if (fault_skip_stage(p.fault, it)) continue;   // debug builds: an injected fault
                     uint8_t* st = smem + s * kStageBytes;
                     mbar_arrive_expect_tx(&full[s], kWBytes + kTBytes + ws_bytes + kNSaBytes);
                     // mode 0: the 128 gate rows, then the 128 up rows of act columns wb*128 .. +127

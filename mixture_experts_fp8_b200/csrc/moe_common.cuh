@@ -18,7 +18,19 @@ namespace moe {
 
 // Bounded waits: a wait that has not finished after this long gives up, records
 // MOE_ERR_TIMEOUT in the status word and lets the kernel leave (no trap, no hang).
-constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// Debug builds (MOE_FAULT_INJECTION): true for the one producer step that an armed
+// MOE_FAULT_SKIP_STAGE drops (CTA 0, first K stage).  Compiled out of the release library.
+__device__ __forceinline__ bool fault_skip_stage(int fault, uint32_t it) {
+#ifdef MOE_FAULT_INJECTION
+    return fault == MOE_FAULT_SKIP_STAGE && blockIdx.x == 0 && it == 0;
+#else
+    (void)fault;
+    (void)it;
+    return false;
+#endif
+}
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;

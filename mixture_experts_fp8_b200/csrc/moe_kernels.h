@@ -86,6 +86,7 @@ struct GemmArgs {
     void* act_s;                // mode 0: [(N/2)/128][a_pad] 4-byte words
     float* out;                 // mode 1: [A, N]
     int32_t* status;
+    int fault;                  // MOE_FAULT_* (acted on only in a MOE_FAULT_INJECTION build)
 };
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);

@@ -84,6 +84,15 @@ int check_config(const moe_config_t* c) {
 
 // Row stride of the stage-major scale arrays: every routed row, plus room for a 128-row tile
 // read starting at a 16-byte-aligned row just before the last row.
+// Fault armed by moe_debug_inject_fault for the next forward on this host thread (debug
+// library only; always MOE_FAULT_NONE in the release library).
+thread_local int t_armed_fault = MOE_FAULT_NONE;
+int take_armed_fault() {
+    const int f = t_armed_fault;
+    t_armed_fault = MOE_FAULT_NONE;
+    return f;
+}
+
 size_t scale_rows_of(size_t A) { return align_up(A + moe::kTileM + 4, 4); }
 
 void layout_of(const moe_config_t* c, moe_workspace_layout_t* L) {
@@ -377,12 +386,14 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     g1.act_q = static_cast<uint8_t*>(at(L.act_q));
     g1.act_s = at(L.act_s);
     g1.status = status;
+    g1.fault = take_armed_fault();
     MOE_CUDA_TRY(mx       ? moe::launch_gemm_mx(g1, tm_x, tm_w13, di.sms, s)
                  : narrow ? moe::launch_gemm_narrow(g1, tm_w13, tm_x, di.sms, s)
                           : moe::launch_gemm(g1, tm_x, tm_w13, di.sms, s));
     MOE_CUDA_TRY(mark(4));
     moe::GemmArgs g2 = g1;
     g2.mode = 1;
+    g2.fault = MOE_FAULT_NONE;
     g2.N = H;
     g2.K = I;
     g2.a_scale = at(L.act_s);
@@ -468,6 +479,17 @@ int moe_selftest_bounded_wait(int32_t* status, uint32_t timeout_us, void* stream
     if (rc) return rc;
     MOE_CUDA_TRY(moe::launch_selftest_wait(status, timeout_us, static_cast<cudaStream_t>(stream)));
     return ok();
+}
+
+int moe_debug_inject_fault(int fault) {
+    if (fault != MOE_FAULT_NONE && fault != MOE_FAULT_SKIP_STAGE)
+        return fail(MOE_ERR_INVALID_ARG, "unknown fault code %d", fault);
+#ifdef MOE_FAULT_INJECTION
+    t_armed_fault = fault;
+    return ok();
+#else
+    return fail(MOE_ERR_UNSUPPORTED, "fault injection needs the debug library (libmoefp8_debug.so)");
+#endif
 }
 
 }  // extern "C"
