@@ -48,7 +48,8 @@ class _Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("num_tokens", "hidden", "inter", "num_experts", "top_k", "routing",
                  "renormalize", "group_count", "k_group", "group_select_mode")] + \
-               [("routed_scaling_factor", ctypes.c_float), ("recipe", ctypes.c_int32)]
+               [("routed_scaling_factor", ctypes.c_float), ("recipe", ctypes.c_int32),
+                ("shared_experts", ctypes.c_int32)]
 
 
 @dataclass
@@ -66,6 +67,12 @@ class Config:
     group_select_mode: int = 0
     routed_scaling_factor: float = 1.0
     recipe: int = 0              # 0 fp32 scale per (row,128); 1 UE8M0 per 32
+    shared_experts: int = 0      # 1: one more expert (index num_experts), every token, weight 1
+
+    @property
+    def slots(self) -> int:
+        """Expert slots per token: the routed top_k plus the shared expert."""
+        return self.top_k + self.shared_experts
 
     @property
     def group(self) -> int:
@@ -79,7 +86,7 @@ class Config:
         return _Cfg(*(int(getattr(self, n)) for n in
                       ("num_tokens", "hidden", "inter", "num_experts", "top_k", "routing",
                        "renormalize", "group_count", "k_group", "group_select_mode")),
-                    float(self.routed_scaling_factor), int(self.recipe))
+                    float(self.routed_scaling_factor), int(self.recipe), int(self.shared_experts))
 
 
 def _load():
@@ -252,8 +259,8 @@ def forward(cfg: Config, x_bf16, w13, w13s, w2, w2s, logits=None, per_expert_sca
     y = np.zeros((n_sel, cfg.hidden), np.uint16)
     act_q = act_s = None
     if want_act:
-        act_q = np.zeros((n_sel, cfg.top_k, cfg.inter), np.uint8)
-        act_s = np.zeros((n_sel, cfg.top_k, cfg.inter // cfg.group), sd)
+        act_q = np.zeros((n_sel, cfg.slots, cfg.inter), np.uint8)
+        act_s = np.zeros((n_sel, cfg.slots, cfg.inter // cfg.group), sd)
     c = cfg.c()
     rc = _load().orc_forward(ctypes.byref(c), *[_p(a) for a in args], _p(tok), n_sel, _p(y),
                              _p(act_q), _p(act_s))

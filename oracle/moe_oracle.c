@@ -48,6 +48,9 @@ typedef struct {
     int32_t group_count, k_group, group_select_mode;
     float routed_scaling_factor;
     int32_t recipe;             /* 0: fp32 scale per (row,128); 1: UE8M0 scale per 32 (MXFP8) */
+    int32_t shared_experts;     /* 0 or 1: one more expert, index num_experts, that every token
+                                   uses with weight 1 ([metrale] run_fp8_grouped_w8a8: the shared
+                                   expert's gate/up/down run in the same grouped steps)          */
 } orc_cfg;
 
 /* ------------------------------------------------------------------------------------------
@@ -229,6 +232,7 @@ int orc_check_cfg(const orc_cfg *c)
     if (c->group_select_mode == 1 && c->num_experts / c->group_count < 2) return ORC_EUNSUPPORTED;
     if (c->routing != 0 && c->routing != 1) return ORC_EINVAL;
     if (c->recipe != 0 && c->recipe != 1) return ORC_EINVAL;
+    if (c->shared_experts != 0 && c->shared_experts != 1) return ORC_EUNSUPPORTED;
     return ORC_OK;
 }
 
@@ -440,12 +444,15 @@ static void expert_mlp_row(const orc_cfg *c, const orc_weights *W, int e, const 
  * output is a contiguous bf16 tensor):
  *   for each token t: route, quantize x_t, run each selected expert, and
  *   y_t = bf16_rn( sum_j w_j * o_j )   (fp64 sum in slot order j = 0..k-1)
+ * With a shared expert (cfg->shared_experts = 1; [metrale] run_fp8_grouped_w8a8 runs it in the
+ * same grouped steps as the routed experts), slot k is expert num_experts with weight 1, added
+ * after the routed slots.
  *
  * `tokens` (n_sel entries) lists which tokens to compute, or is NULL for all of them; y and
  * the per-token outputs are indexed by position in that list.  When topk_idx_in is non-NULL
  * the routing is taken from it and topk_w_in (the custom routing function path of [MindIE]);
  * otherwise it is computed from the logits.  act_q/act_s (optional) receive each slot's
- * requantized SwiGLU product, [n_sel, k, I] and [n_sel, k, I/g].
+ * requantized SwiGLU product, [n_sel, k + S, I] and [n_sel, k + S, I/g] (S = shared_experts).
  * ---------------------------------------------------------------------------------------- */
 int orc_forward(const orc_cfg *c, const uint16_t *x, const float *logits,
                 const float *per_expert_scale, const int32_t *topk_idx_in,
@@ -454,6 +461,7 @@ int orc_forward(const orc_cfg *c, const uint16_t *x, const float *logits,
                 const int32_t *tokens, int n_sel, uint16_t *y, uint8_t *act_q, void *act_s)
 {
     const int H = c->hidden, I = c->inter, K = c->top_k, g = c->recipe == 0 ? 128 : 32;
+    const int KT = K + c->shared_experts;             /* slots per token */
     const size_t sb = scale_bytes(c->recipe);
     orc_weights W = {w13, w13s, w2, w2s, b13, b2};
     int rc = orc_check_cfg(c);
@@ -464,8 +472,8 @@ int orc_forward(const orc_cfg *c, const uint16_t *x, const float *logits,
 #pragma omp parallel for schedule(dynamic, 1)
     for (int p = 0; p < n_sel; p++) {
         const int t = tokens ? tokens[p] : p;
-        int32_t ids[256];
-        float wts[256];
+        int32_t ids[257];
+        float wts[257];
         float *xf = (float *)malloc(sizeof(float) * (size_t)H);
         uint8_t *xq = (uint8_t *)malloc((size_t)H);
         void *xs = malloc(sb * (size_t)(H / g));
@@ -480,11 +488,15 @@ int orc_forward(const orc_cfg *c, const uint16_t *x, const float *logits,
         } else {
             route_token(c, logits + (size_t)t * c->num_experts, per_expert_scale, ids, wts);
         }
+        if (c->shared_experts) {                       /* the shared expert: slot k, weight 1 */
+            ids[K] = c->num_experts;
+            wts[K] = 1.0f;
+        }
         for (int h = 0; h < H; h++) xf[h] = bf16_to_f32(x[(size_t)t * H + h]);
         orc_quant_row(xf, H, c->recipe, xq, xs);
-        for (int j = 0; j < K; j++) {
-            uint8_t *aq = act_q ? act_q + ((size_t)p * K + j) * I : NULL;
-            void *as = act_s ? (uint8_t *)act_s + ((size_t)p * K + j) * (I / g) * sb : NULL;
+        for (int j = 0; j < KT; j++) {
+            uint8_t *aq = act_q ? act_q + ((size_t)p * KT + j) * I : NULL;
+            void *as = act_s ? (uint8_t *)act_s + ((size_t)p * KT + j) * (I / g) * sb : NULL;
             expert_mlp_row(c, &W, ids[j], xq, xs, o, aq, as);
             for (int h = 0; h < H; h++) acc[h] += (double)wts[j] * o[h];
         }
@@ -504,7 +516,8 @@ int orc_forward_permuted(const orc_cfg *c, const uint16_t *x, const float *logit
                          const uint8_t *w2, const void *w2s, const uint16_t *b13,
                          const uint16_t *b2, uint16_t *y)
 {
-    const int T = c->num_tokens, H = c->hidden, K = c->top_k, E = c->num_experts;
+    const int T = c->num_tokens, H = c->hidden, E = c->num_experts + c->shared_experts;
+    const int K = c->top_k + c->shared_experts;   /* slots per token, the shared one last */
     const int g = c->recipe == 0 ? 128 : 32, A = T * K;
     const size_t sb = scale_bytes(c->recipe);
     orc_weights W = {w13, w13s, w2, w2s, b13, b2};
@@ -520,7 +533,23 @@ int orc_forward_permuted(const orc_cfg *c, const uint16_t *x, const float *logit
     row_src = (int32_t *)malloc(sizeof(int32_t) * (size_t)A);
     row_of = (int32_t *)malloc(sizeof(int32_t) * (size_t)A);
     o = (double *)malloc(sizeof(double) * (size_t)A * H);
-    orc_route(c, logits, per_expert_scale, idx, wts, NULL);
+    {
+        const int k = c->top_k;
+        int32_t *ridx = (int32_t *)malloc(sizeof(int32_t) * (size_t)T * k);
+        float *rw = (float *)malloc(sizeof(float) * (size_t)T * k);
+        orc_route(c, logits, per_expert_scale, ridx, rw, NULL);
+        for (int t = 0; t < T; t++) {
+            for (int j = 0; j < k; j++) {
+                idx[t * K + j] = ridx[t * k + j];
+                wts[t * K + j] = rw[t * k + j];
+            }
+            if (c->shared_experts) {
+                idx[t * K + k] = c->num_experts;
+                wts[t * K + k] = 1.0f;
+            }
+        }
+        free(ridx); free(rw);
+    }
     orc_permute(T, K, E, idx, counts, offsets, row_src, row_of);
 
     /* mlp: expert by expert over its contiguous rows */

@@ -57,6 +57,7 @@ class Shape:
     zipf_s: float = 0.0              # > 0: add ln p_e, p_e ~ rank^-s
     per_expert_scale: bool = False   # draw per_expert_scale ~ U(0.5, 1.5)
     biases: bool = False             # draw w13_bias / w2_bias ~ N(0, 0.02) in bf16
+    shared_experts: int = 0          # 1: weights for one more expert, which every token uses
 
     @property
     def group(self) -> int:
@@ -68,7 +69,8 @@ class Shape:
                     num_experts=self.num_experts, top_k=self.top_k, routing=self.routing,
                     renormalize=self.renormalize, group_count=self.group_count,
                     k_group=self.k_group, group_select_mode=self.group_select_mode,
-                    routed_scaling_factor=self.routed_scaling_factor, recipe=self.recipe)
+                    routed_scaling_factor=self.routed_scaling_factor, recipe=self.recipe,
+                    shared_experts=self.shared_experts)
 
     def with_tokens(self, n: int) -> "Shape":
         return replace(self, num_tokens=n)
@@ -133,7 +135,7 @@ class Problem:
     x: torch.Tensor                      # bf16 [T,H]
     logits: torch.Tensor                 # fp32 [T,E]
     per_expert_scale: torch.Tensor | None
-    w13: torch.Tensor                    # uint8 [E,H,2I]
+    w13: torch.Tensor                    # uint8 [E,H,2I]  (E + 1 experts with a shared expert)
     w13_scale: torch.Tensor              # fp32 [E,H/128,2I] | uint8 [E,H/32,2I]
     w2: torch.Tensor                     # uint8 [E,I,H]
     w2_scale: torch.Tensor               # fp32 [E,I/128,H]  | uint8 [E,I/32,H]
@@ -163,8 +165,10 @@ class Problem:
 
 
 def make_weights(shape: Shape, device="cpu"):
-    """Per-expert fp32 N(0, 1/sqrt(K)) weights, prepared as codes + block scales."""
-    E, H, I, r = shape.num_experts, shape.hidden, shape.inter, shape.recipe
+    """Per-expert fp32 N(0, 1/sqrt(K)) weights, prepared as codes + block scales; the shared
+    expert, if any, is expert index num_experts (drawn from its own seed, so the routed
+    experts' weights do not depend on it)."""
+    E, H, I, r = shape.num_experts + shape.shared_experts, shape.hidden, shape.inter, shape.recipe
     g = shape.group
     sdt = torch.float32 if r == 0 else torch.uint8
     w13 = torch.empty((E, H, 2 * I), dtype=torch.uint8, device=device)
@@ -207,6 +211,9 @@ def make_problem(name_or_shape, device="cpu", num_tokens: int | None = None) -> 
         E, H, I = shape.num_experts, shape.hidden, shape.inter
         b13 = _randn((E, 2 * I), 0.02, device, shape.seed, _B13).to(torch.bfloat16)
         b2 = _randn((E, H), 0.02, device, shape.seed, _B2).to(torch.bfloat16)
+        if shape.shared_experts:                     # the shared expert's rows, own seed
+            b13 = torch.cat([b13, _randn((1, 2 * I), 0.02, device, shape.seed, _B13, E).to(torch.bfloat16)])
+            b2 = torch.cat([b2, _randn((1, H), 0.02, device, shape.seed, _B2, E).to(torch.bfloat16)])
     return Problem(shape, x, logits, pes, w13, w13s, w2, w2s, b13, b2)
 
 
