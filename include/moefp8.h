@@ -61,6 +61,12 @@ extern "C" {
  *   recipe             0 = E4M3 with an fp32 scale per (row, 128-element block) for
  *                          activations and per (output column, 128-deep K block) for weights
  *                      1 = MXFP8: E4M3 with a UE8M0 power-of-two scale per 32 elements
+ *   shared_experts     0, or 1: one more expert, index num_experts, that every token uses with
+ *                      weight 1 after its top_k routed experts ("metrale_model_layers
+ *                      fp8_grouped_tc_w8a8.rs", run_fp8_grouped_w8a8: the shared expert's
+ *                      gate/up and down run in the same grouped steps).  The weight and bias
+ *                      tensors then hold num_experts + 1 experts, the shared one last; the
+ *                      router still selects among num_experts.
  * Limits (MOE_ERR_UNSUPPORTED): hidden % 128, inter % 128, num_experts <= 256,
  * num_experts % group_count, k_group in [1, group_count], top_k <= k_group * experts per
  * group, group_select_mode 1 needs >= 2 experts per group.  ("MATE Mega MoE", Current Limits
@@ -73,10 +79,12 @@ typedef struct {
     int32_t group_count, k_group, group_select_mode;
     float routed_scaling_factor;
     int32_t recipe;
+    int32_t shared_experts;
 } moe_config_t;
 
 /* Byte offsets of the regions inside a forward workspace (for tests and diagnostics).
- * A = num_tokens * top_k routed rows.  Scales are stored K-block-major: one 4-byte word per
+ * S = shared_experts, k' = top_k + S expert slots per token (slot top_k is the shared
+ * expert), E' = num_experts + S, A = num_tokens * k' rows.  Scales are stored K-block-major: one 4-byte word per
  * (128-column block, row) with a row stride of scale_rows words; the word is the fp32 scale
  * (recipe 0) or the four UE8M0 bytes of the block's four 32-column groups, lowest group in the
  * lowest byte (recipe 1).  All offsets are multiples of 1024. */
@@ -84,11 +92,11 @@ typedef struct {
     size_t status;       /* int32 status word (MOE_OK or a device MOE_ERR_*)             */
     size_t topk_idx;     /* int32 [T, k]   routing computed by moe_forward               */
     size_t topk_weights; /* fp32  [T, k]                                                 */
-    size_t counts;       /* int32 [E]      routed rows per expert                        */
-    size_t offsets;      /* int32 [E + 1]  first permuted row of each expert             */
-    size_t tile_start;   /* int32 [E + 1]  first 128-row M tile of each expert           */
-    size_t row_src;      /* int32 [A]      permuted row r came from routed row t*k + j   */
-    size_t row_of;       /* int32 [T, k]   permuted row of routed row (t, j)             */
+    size_t counts;       /* int32 [E']     rows per expert                               */
+    size_t offsets;      /* int32 [E' + 1] first permuted row of each expert             */
+    size_t tile_start;   /* int32 [E' + 1] first 128-row M tile of each expert           */
+    size_t row_src;      /* int32 [A]      permuted row r came from slot row t*k' + j    */
+    size_t row_of;       /* int32 [T, k']  permuted row of slot (t, j)                   */
     size_t hist;         /* int32 [chunks, E] per-chunk expert histograms                */
     size_t xq;           /* E4M3  [A, H]   quantized activations in permuted order       */
     size_t xs;           /* word  [H/128, scale_rows]                                    */
@@ -118,6 +126,7 @@ int moe_transformed_weights_size(const moe_config_t *cfg, size_t *w13_bytes, siz
 
 /* Re-lay the grouped FP8 expert weights for the forward ("MATE Mega MoE", Typical Flow step 2
  * and transform_weights_for_mega_moe).  Runs once, offline; deterministic and re-runnable.
+ * (E below is num_experts + shared_experts: the shared expert's tensors come last.)
  *   w13        device, E4M3 codes [E, H, 2I] (K rows x N columns; columns 0:I gate, I:2I up)
  *   w13_scale  device, recipe 0: fp32 [E, H/128, 2I]; recipe 1: UE8M0 bytes [E, H/32, 2I]
  *   w2         device, E4M3 codes [E, I, H]
@@ -158,10 +167,11 @@ int moe_route(const moe_config_t *cfg, const float *router_logits, const float *
  *                                           router_logits and topk_idx must be non-NULL.
  *                                           The k ids of a token must be distinct, in [0, E).
  *   w13_t .. w2s_t    device, from moe_transform_weights with the same cfg fields
- *   w13_bias          device bf16 [E, 2I] or NULL (16-byte aligned)
- *   w2_bias           device bf16 [E, H] or NULL (16-byte aligned)
+ *   w13_bias          device bf16 [E', 2I] or NULL (16-byte aligned; E' = num_experts + shared_experts)
+ *   w2_bias           device bf16 [E', H] or NULL (16-byte aligned)
  *   y                 device bf16 [T, H], contiguous; out
- *   expert_counts     device int32 [E] or NULL; out: rows routed to each expert
+ *   expert_counts     device int32 [E'] or NULL; out: rows routed to each expert (the shared
+ *                     expert's count is num_tokens)
  *   workspace         device, >= moe_workspace_size bytes, 1024-byte aligned; scratch owned by
  *                     the caller; must not be shared by calls in flight at the same time
  * A row's output bits do not depend on the other rows of the batch. */

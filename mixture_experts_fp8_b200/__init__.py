@@ -51,7 +51,8 @@ class _Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("num_tokens", "hidden", "inter", "num_experts", "top_k", "routing",
                  "renormalize", "group_count", "k_group", "group_select_mode")] + \
-               [("routed_scaling_factor", ctypes.c_float), ("recipe", ctypes.c_int32)]
+               [("routed_scaling_factor", ctypes.c_float), ("recipe", ctypes.c_int32),
+                ("shared_experts", ctypes.c_int32)]
 
 
 _LAYOUT_FIELDS = ("status", "topk_idx", "topk_weights", "counts", "offsets", "tile_start",
@@ -66,7 +67,8 @@ class _Layout(ctypes.Structure):
 @dataclass
 class Config:
     """One problem (moe_config_t).  routing: 0 softmax, 1 sigmoid; recipe: 0 fp32 scale per
-    (row, 128), 1 MXFP8 (UE8M0 per 32)."""
+    (row, 128), 1 MXFP8 (UE8M0 per 32); shared_experts: 1 adds an expert (index num_experts)
+    that every token uses with weight 1."""
     num_tokens: int
     hidden: int
     inter: int
@@ -79,13 +81,14 @@ class Config:
     group_select_mode: int = 0
     routed_scaling_factor: float = 1.0
     recipe: int = 0
+    shared_experts: int = 0
 
     def c(self) -> _Cfg:
         d = asdict(self)
         return _Cfg(*(int(d[n]) for n in ("num_tokens", "hidden", "inter", "num_experts", "top_k",
                                           "routing", "renormalize", "group_count", "k_group",
                                           "group_select_mode")),
-                    float(d["routed_scaling_factor"]), int(d["recipe"]))
+                    float(d["routed_scaling_factor"]), int(d["recipe"]), int(d["shared_experts"]))
 
     @property
     def group(self) -> int:

@@ -72,8 +72,8 @@ struct L {
     static constexpr uint32_t misc = amax_bar + 16;      // tmem holder, abort flag
     static constexpr uint32_t amax = misc + 16;          // float [2 buffers][4 quarters][128 rows]
     static constexpr uint32_t tstart = amax + 2 * 4 * 128 * 4;
-    static constexpr uint32_t off = tstart + (MOE_MAX_EXPERTS + 1) * 4;
-    static constexpr uint32_t end = off + (MOE_MAX_EXPERTS + 1) * 4;
+    static constexpr uint32_t off = tstart + (MOE_MAX_EXPERTS + 2) * 4;   // experts + a shared one, + 1
+    static constexpr uint32_t end = off + (MOE_MAX_EXPERTS + 2) * 4;   // experts + a shared one, + 1
 };
 static_assert(kWsBytes + kSaBytes <= kScaleSlot, "scale slot");
 constexpr uint32_t kSmemBytes = L::end + 1024;   // + slack to align the base to 1024 bytes

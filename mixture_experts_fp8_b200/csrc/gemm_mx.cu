@@ -48,8 +48,8 @@ struct XL {
     static constexpr uint32_t nbars = 3 * kXStages + 5;   // full, sfready, empty, tfull[2], tempty[2], drain
     static constexpr uint32_t misc = bars + nbars * 8;
     static constexpr uint32_t tstart = misc + 16;
-    static constexpr uint32_t off = tstart + (MOE_MAX_EXPERTS + 1) * 4;
-    static constexpr uint32_t end = off + (MOE_MAX_EXPERTS + 1) * 4;
+    static constexpr uint32_t off = tstart + (MOE_MAX_EXPERTS + 2) * 4;   // experts + a shared one, + 1
+    static constexpr uint32_t end = off + (MOE_MAX_EXPERTS + 2) * 4;   // experts + a shared one, + 1
 };
 static_assert(kXStage % 1024 == 0, "stage alignment");
 constexpr uint32_t kXSmemBytes = XL::end + 1024;

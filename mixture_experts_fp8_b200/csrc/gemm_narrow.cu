@@ -53,8 +53,8 @@ struct NL {
     static constexpr uint32_t misc = bars + nbars * 8;               // tmem holder, abort flag
     static constexpr uint32_t amax = misc + 16;                      // float [2][4 quads][kNT]
     static constexpr uint32_t ustart = amax + 2 * 4 * kNT * 4;       // int [E + 1] unit prefix
-    static constexpr uint32_t off = ustart + (MOE_MAX_EXPERTS + 1) * 4;
-    static constexpr uint32_t end = off + (MOE_MAX_EXPERTS + 1) * 4;
+    static constexpr uint32_t off = ustart + (MOE_MAX_EXPERTS + 2) * 4;   // experts + a shared one, + 1
+    static constexpr uint32_t end = off + (MOE_MAX_EXPERTS + 2) * 4;   // experts + a shared one, + 1
 };
 static_assert(NL::sa + kNSaBytes <= kStageBytes, "stage layout");
 static_assert(kStageBytes % 1024 == 0, "stage alignment");

@@ -36,8 +36,10 @@ struct RouteArgs {
     int32_t* status;            // cleared to MOE_OK by the first thread when non-null
 };
 
+// Rows r = t * KT + j of the permutation: slot j < k is routed to idx[t * k + j]; slot k (when
+// KT > k) is the shared expert, index E, which every token uses.
 struct PermuteArgs {
-    const int32_t* idx;         // [A]
+    const int32_t* idx;         // [T, k] routed expert ids
     int32_t* hist;              // [chunks, E]  (per-chunk counts, then exclusive bases)
     int32_t* counts;            // [E]
     int32_t* offsets;           // [E + 1]
@@ -46,8 +48,17 @@ struct PermuteArgs {
     int32_t* row_of;            // [A]
     int32_t* expert_counts;     // [E] or null (caller's copy)
     int32_t* status;
-    int A, E, chunks, chunk;    // chunk = routed rows per chunk
+    int A, E, chunks, chunk;    // A = T * KT rows; E routed experts; chunk = rows per chunk
+    int T, k, KT;
 };
+
+// The expert of permutation row r: a routed expert id (range-checked by the callers), or
+// kSharedSlot for the shared expert's slot.
+constexpr int kSharedSlot = -2;
+__host__ __device__ inline int slot_expert(const PermuteArgs& a, int r) {
+    const int t = r / a.KT, j = r - t * a.KT;
+    return j < a.k ? a.idx[static_cast<size_t>(t) * a.k + j] : kSharedSlot;
+}
 
 struct QuantArgs {
     const __nv_bfloat16* x;     // [T, H]
@@ -60,10 +71,10 @@ struct QuantArgs {
 
 struct CombineArgs {
     const float* o;             // [A, H]
-    const int32_t* row_of;      // [T, K]
-    const float* w;             // [T, K]
+    const int32_t* row_of;      // [T, K]  (K slots per token)
+    const float* w;             // [T, k]  routing weights of the k routed slots
     __nv_bfloat16* y;           // [T, H]
-    int T, H, K;
+    int T, H, K, k;             // slots j >= k (the shared expert's) have weight 1
 };
 
 struct TransformArgs {

@@ -62,6 +62,8 @@ int check_config(const moe_config_t* c) {
     if (c->inter % 128) return fail(MOE_ERR_UNSUPPORTED, "inter (%d) must be a multiple of 128", c->inter);
     if (c->num_experts > MOE_MAX_EXPERTS)
         return fail(MOE_ERR_UNSUPPORTED, "num_experts (%d) exceeds %d", c->num_experts, MOE_MAX_EXPERTS);
+    if (c->shared_experts != 0 && c->shared_experts != 1)
+        return fail(MOE_ERR_UNSUPPORTED, "shared_experts must be 0 or 1, got %d", c->shared_experts);
     if (c->group_count < 1 || c->num_experts % c->group_count)
         return fail(MOE_ERR_UNSUPPORTED, "num_experts (%d) must be divisible by group_count (%d)", c->num_experts,
                     c->group_count);
@@ -75,9 +77,9 @@ int check_config(const moe_config_t* c) {
         return fail(MOE_ERR_INVALID_ARG, "group_select_mode must be 0 or 1, got %d", c->group_select_mode);
     if (c->group_select_mode == 1 && per_group < 2)
         return fail(MOE_ERR_UNSUPPORTED, "group_select_mode 1 needs at least 2 experts per group");
-    const long long A = 1LL * c->num_tokens * c->top_k;
-    if (A > (1LL << 30) || 1LL * c->num_experts * 2 * c->inter > (1LL << 30) ||
-        1LL * c->num_experts * c->hidden > (1LL << 30))
+    const long long A = 1LL * c->num_tokens * (c->top_k + c->shared_experts);
+    const long long ET = c->num_experts + c->shared_experts;
+    if (A > (1LL << 30) || ET * 2 * c->inter > (1LL << 30) || ET * c->hidden > (1LL << 30))
         return fail(MOE_ERR_UNSUPPORTED, "problem too large for 32-bit row indices");
     return MOE_OK;
 }
@@ -96,8 +98,11 @@ int take_armed_fault() {
 size_t scale_rows_of(size_t A) { return align_up(A + moe::kTileM + 4, 4); }
 
 void layout_of(const moe_config_t* c, moe_workspace_layout_t* L) {
+    // k routed slots per token (the router's output), KT = k + shared slots, E routed experts,
+    // ET = E + shared, A = T * KT permuted rows
     const size_t T = c->num_tokens, K = c->top_k, E = c->num_experts, H = c->hidden, I = c->inter;
-    const size_t A = T * K, SR = scale_rows_of(A);
+    const size_t KT = K + c->shared_experts, ET = E + c->shared_experts;
+    const size_t A = T * KT, SR = scale_rows_of(A);
     const size_t chunks = moe::permute_chunks(static_cast<long long>(A));
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -106,11 +111,11 @@ void layout_of(const moe_config_t* c, moe_workspace_layout_t* L) {
         return o;
     };
     L->status = take(16);
-    L->topk_idx = take(4 * A);
-    L->topk_weights = take(4 * A);
-    L->counts = take(4 * E);
-    L->offsets = take(4 * (E + 1));
-    L->tile_start = take(4 * (E + 1));
+    L->topk_idx = take(4 * T * K);
+    L->topk_weights = take(4 * T * K);
+    L->counts = take(4 * ET);
+    L->offsets = take(4 * (ET + 1));
+    L->tile_start = take(4 * (ET + 1));
     L->row_src = take(4 * A);
     L->row_of = take(4 * A);
     L->hist = take(4 * chunks * E);
@@ -229,7 +234,7 @@ int moe_transformed_weights_size(const moe_config_t* cfg, size_t* w13_bytes, siz
     int rc = check_config(cfg);
     if (rc) return rc;
     if (!w13_bytes || !w13s_bytes || !w2_bytes || !w2s_bytes) return fail(MOE_ERR_INVALID_ARG, "NULL size pointer");
-    const size_t E = cfg->num_experts, H = cfg->hidden, I = cfg->inter;
+    const size_t E = cfg->num_experts + cfg->shared_experts, H = cfg->hidden, I = cfg->inter;
     *w13_bytes = E * 2 * I * H;
     *w13s_bytes = E * (H / 128) * 2 * I * 4;
     *w2_bytes = E * H * I;
@@ -250,7 +255,7 @@ int moe_transform_weights(const moe_config_t* cfg, const void* w13, const void* 
     if ((rc = device_info(&di))) return rc;
     moe::TransformArgs a{static_cast<const uint8_t*>(w13), w13_scale, static_cast<const uint8_t*>(w2), w2_scale,
                          static_cast<uint8_t*>(w13_t), w13s_t, static_cast<uint8_t*>(w2_t), w2s_t,
-                         cfg->num_experts, cfg->hidden, cfg->inter, cfg->recipe};
+                         cfg->num_experts + cfg->shared_experts, cfg->hidden, cfg->inter, cfg->recipe};
     MOE_CUDA_TRY(moe::launch_transform(a, static_cast<cudaStream_t>(stream)));
     return ok();
 }
@@ -315,8 +320,10 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     DeviceInfo di;
     if ((rc = device_info(&di))) return rc;
 
+    // K routed slots per token, KT with the shared expert's slot; E routed experts, ET in all
     const int T = cfg->num_tokens, K = cfg->top_k, E = cfg->num_experts, H = cfg->hidden, I = cfg->inter;
-    const int A = T * K;
+    const int KT = K + cfg->shared_experts, ET = E + cfg->shared_experts;
+    const int A = T * KT;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
     int32_t* status = static_cast<int32_t*>(at(L.status));
@@ -329,15 +336,15 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     // take the swap-AB kernels, weights as the M operand, else the wide kernels; both compute every
     // row with the same operations, so the choice does not change bits.
     const bool mx = cfg->recipe == 1;
-    const bool narrow = !mx && A <= moe::kNarrowRowsPerExpert * E;
+    const bool narrow = !mx && A <= moe::kNarrowRowsPerExpert * ET;
     CUtensorMap tm_x, tm_w13, tm_act, tm_w2;
     const uint32_t tok_box = narrow ? 16 : moe::kTileM;
     const uint32_t w13_box = mx ? 128 : narrow ? moe::kTileN : moe::gemm_weight_box(0);
     const uint32_t w2_box = mx ? 128 : narrow ? moe::kTileN : moe::gemm_weight_box(1);
     if ((rc = make_kmajor_map(&tm_x, at(L.xq), A, H, tok_box))) return rc;
-    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(E) * 2 * I, H, w13_box))) return rc;
+    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(ET) * 2 * I, H, w13_box))) return rc;
     if ((rc = make_kmajor_map(&tm_act, at(L.act_q), A, I, tok_box))) return rc;
-    if ((rc = make_kmajor_map(&tm_w2, w2_t, static_cast<uint64_t>(E) * H, I, w2_box))) return rc;
+    if ((rc = make_kmajor_map(&tm_w2, w2_t, static_cast<uint64_t>(ET) * H, I, w2_box))) return rc;
 
     cudaEvent_t* ev = nullptr;
     if (prof && (rc = prof_next(prof, &ev))) return rc;
@@ -351,7 +358,7 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     moe::PermuteArgs pa{idx, static_cast<int32_t*>(at(L.hist)), static_cast<int32_t*>(at(L.counts)),
                         static_cast<int32_t*>(at(L.offsets)), static_cast<int32_t*>(at(L.tile_start)),
                         static_cast<int32_t*>(at(L.row_src)), static_cast<int32_t*>(at(L.row_of)), expert_counts,
-                        status, A, E, moe::permute_chunks(A), moe::permute_chunk_rows(A)};
+                        status, A, E, moe::permute_chunks(A), moe::permute_chunk_rows(A), T, K, KT};
     MOE_CUDA_TRY(mark(0));
     // The first kernel of the forward clears the status word: the router when it runs, else the
     // small-batch permutation; a memset otherwise.
@@ -366,7 +373,7 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     else MOE_CUDA_TRY(moe::launch_permute(pa, s));
     MOE_CUDA_TRY(mark(2));
     moe::QuantArgs qa{static_cast<const __nv_bfloat16*>(hidden_states), static_cast<const int32_t*>(at(L.row_of)),
-                      static_cast<uint8_t*>(at(L.xq)), at(L.xs), status, T, H, K, cfg->recipe,
+                      static_cast<uint8_t*>(at(L.xq)), at(L.xs), status, T, H, KT, cfg->recipe,
                       static_cast<int>(L.scale_rows)};
     MOE_CUDA_TRY(moe::launch_quant(qa, s));
     MOE_CUDA_TRY(mark(3));
@@ -375,7 +382,7 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     g1.recipe = cfg->recipe;
     g1.N = 2 * I;
     g1.K = H;
-    g1.E = E;
+    g1.E = ET;
     g1.A = A;
     g1.a_pad = static_cast<int>(L.scale_rows);
     g1.offsets = static_cast<const int32_t*>(at(L.offsets));
@@ -407,7 +414,7 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
                           : moe::launch_gemm(g2, tm_act, tm_w2, di.sms, s));
     MOE_CUDA_TRY(mark(5));
     moe::CombineArgs ca{static_cast<const float*>(at(L.o)), static_cast<const int32_t*>(at(L.row_of)), wts,
-                        static_cast<__nv_bfloat16*>(y), T, H, K};
+                        static_cast<__nv_bfloat16*>(y), T, H, KT, K};
     MOE_CUDA_TRY(moe::launch_combine(ca, s));
     MOE_CUDA_TRY(mark(6));
     return ok();

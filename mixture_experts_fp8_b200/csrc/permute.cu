@@ -1,9 +1,11 @@
 // permute.cu -- stable permutation of the routed rows into expert-contiguous order.
 //
 // "MindIE-SD Fused MoE", execution flow: dispatch reorders tokens by expert and counts each
-// expert's tokens; combine restores token order.  Routed row a = t*k + j; inside an expert,
-// rows keep ascending a (hence ascending token).  Three launches, no global atomics, so the
-// result is the same bits on every run:
+// expert's tokens; combine restores token order.  Slot row a = t*KT + j (slot j < k routed,
+// slot k the shared expert when there is one); inside an expert, rows keep ascending a (hence
+// ascending token).  The shared expert (index E) holds every token, so its count (T) and its
+// rows (token order) are known without counting; it is appended after the routed experts.
+// Three launches, no global atomics, so the result is the same bits on every run:
 //   1. k_hist     per-chunk expert histograms (a chunk is a multiple of kPermuteChunk routed
 //                 rows, sized so that there are at most kMaxPermuteChunks chunks)
 //   2. k_scan     per-expert exclusive bases across chunks, counts, offsets = exclusive scan,
@@ -24,7 +26,8 @@ __global__ void __launch_bounds__(256) k_hist(PermuteArgs a) {
     const int begin = blockIdx.x * a.chunk;
     const int end = min(a.A, begin + a.chunk);
     for (int r = begin + threadIdx.x; r < end; r += blockDim.x) {
-        const int e = a.idx[r];
+        const int e = slot_expert(a, r);
+        if (e == kSharedSlot) continue;
         if (e >= 0 && e < a.E) atomicAdd(&cnt[e], 1);
         else set_status(a.status, MOE_ERR_BOUNDS);
     }
@@ -60,6 +63,14 @@ __device__ int block_exclusive_scan_256(int v, int* tmp) {
     return excl;
 }
 
+// The shared expert (index E): every token, in token order, after the routed experts' rows.
+__device__ __forceinline__ void append_shared(const PermuteArgs& a, int off, int ts) {
+    a.counts[a.E] = a.T;
+    a.offsets[a.E + 1] = off + a.T;
+    a.tile_start[a.E + 1] = ts + (a.T + kTileM - 1) / kTileM;
+    if (a.expert_counts) a.expert_counts[a.E] = a.T;
+}
+
 __global__ void __launch_bounds__(256) k_scan(PermuteArgs a) {
     __shared__ int tmp[16];
     pdl_wait_then_release();
@@ -89,6 +100,7 @@ __global__ void __launch_bounds__(256) k_scan(PermuteArgs a) {
     if (e == a.E - 1) {
         a.offsets[a.E] = off + cnt;
         a.tile_start[a.E] = ts + mt;
+        if (a.KT > a.k) append_shared(a, off + cnt, ts + mt);
     }
 }
 
@@ -101,20 +113,26 @@ __global__ void __launch_bounds__(32) k_scatter(PermuteArgs a) {
     const int end = min(a.A, begin + a.chunk);
     for (int e = lane; e < a.E; e += 32)
         base[e] = a.offsets[e] + a.hist[static_cast<size_t>(blockIdx.x) * a.E + e];
+    const int shared_base = a.KT > a.k ? a.offsets[a.E] : 0;
     __syncwarp();
     for (int p0 = begin; p0 < end; p0 += kPermuteChunk) {
         int ids[kBatches];                              // the next 256 ids, loaded at once
 #pragma unroll
         for (int b = 0; b < kBatches; ++b) {
             const int r = p0 + 32 * b + lane;
-            ids[b] = r < end ? a.idx[r] : -1;
+            ids[b] = r < end ? slot_expert(a, r) : -1;
         }
 #pragma unroll
         for (int b = 0; b < kBatches; ++b) {
             const int r = p0 + 32 * b + lane;
             const bool valid = r < end;
             int e = ids[b];
-            if (e >= a.E) e = -1;                       // reported by k_hist
+            if (valid && e == kSharedSlot) {            // the shared expert: token order
+                const int dst = shared_base + r / a.KT;
+                a.row_src[dst] = r;
+                a.row_of[r] = dst;
+            }
+            if (e >= a.E) e = -1;                       // reported by k_hist; shared slots too
             const uint32_t active = __ballot_sync(0xffffffffu, valid && e >= 0);
             const uint32_t peers = __match_any_sync(0xffffffffu, e);
             const uint32_t mine = peers & active;
@@ -141,6 +159,7 @@ constexpr size_t kSmallSmem = kSmallRows * 4 + kSmallWarps * MOE_MAX_EXPERTS * 4
 
 __global__ void __launch_bounds__(kSmallWarps * 32) k_permute_small(PermuteArgs pa, int clear_status) {
     extern __shared__ uint8_t sm[];
+    __shared__ int s_shared_base;                      // first row of the shared expert
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int* ids = reinterpret_cast<int*>(sm);
     int* hist = ids + kSmallRows;                      // [warp][E]
@@ -149,12 +168,13 @@ __global__ void __launch_bounds__(kSmallWarps * 32) k_permute_small(PermuteArgs 
     pdl_wait_then_release();
     if (clear_status && threadIdx.x == 0 && pa.status) *pa.status = MOE_OK;
     for (int i = threadIdx.x; i < kSmallWarps * E; i += blockDim.x) hist[i] = 0;
-    for (int r = threadIdx.x; r < A; r += blockDim.x) ids[r] = pa.idx[r];
+    for (int r = threadIdx.x; r < A; r += blockDim.x) ids[r] = slot_expert(pa, r);
     __syncthreads();
     const int C = ((A + kSmallWarps - 1) / kSmallWarps + 31) / 32 * 32;
     const int begin = warp * C, end = min(A, begin + C);
     for (int r = begin + lane; r < end; r += 32) {
         const int e = ids[r];
+        if (e == kSharedSlot) continue;
         if (e >= 0 && e < E) atomicAdd(&hist[warp * E + e], 1);
         else set_status(pa.status, MOE_ERR_BOUNDS);
     }
@@ -206,6 +226,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32) k_permute_small(PermuteArgs 
         if (lane == 31) {
             pa.offsets[E] = base;
             pa.tile_start[E] = mbase;
+            s_shared_base = base;
+            if (pa.KT > pa.k) append_shared(pa, base, mbase);
         }
     }
     __syncthreads();
@@ -215,6 +237,11 @@ __global__ void __launch_bounds__(kSmallWarps * 32) k_permute_small(PermuteArgs 
         const int r = r0 + lane;
         const bool valid = r < end;
         int e = valid ? ids[r] : -1;
+        if (valid && e == kSharedSlot) {                // the shared expert: token order
+            const int dst = s_shared_base + r / pa.KT;
+            pa.row_src[dst] = r;
+            pa.row_of[r] = dst;
+        }
         if (e >= E) e = -1;
         const uint32_t active = __ballot_sync(0xffffffffu, valid && e >= 0);
         const uint32_t peers = __match_any_sync(0xffffffffu, e);

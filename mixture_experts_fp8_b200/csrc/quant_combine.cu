@@ -8,7 +8,8 @@
 //   recipe 0: s = amax / 448 (IEEE division), q = e4m3_rn_satfinite(x / s); amax 0 -> s = 1
 //   recipe 1: s = 2^e, e the smallest with amax <= 448 * 2^e; byte e + 127; q = e4m3(x * 2^-e)
 //
-// k_combine: y[t] = bf16_rn( sum_j w[t,j] * o[row_of[t,j]] ), fp32, fixed slot order, no
+// k_combine: y[t] = bf16_rn( sum_j w[t,j] * o[row_of[t,j]] ), fp32, fixed slot order (the
+// shared expert's slot, if any, last with weight 1), no
 // atomics ("MindIE-SD Fused MoE", execution flow: combine; "MATE Mega MoE", Current Limits:
 // contiguous bf16 output).
 #include "moe_common.cuh"
@@ -78,15 +79,15 @@ cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s) {
 // Grid (token, column block): thread i of block (t, cb) handles float4 column cb * 256 + i, so
 // every routed row's loads are in flight at once.
 __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
-    __shared__ int s_row[MOE_MAX_EXPERTS];
-    __shared__ float s_w[MOE_MAX_EXPERTS];
+    __shared__ int s_row[MOE_MAX_EXPERTS + 1];
+    __shared__ float s_w[MOE_MAX_EXPERTS + 1];
     pdl_wait_then_release();
     const int t = blockIdx.x;
     const int A = a.T * a.K;
     for (int j = threadIdx.x; j < a.K; j += blockDim.x) {
         int r = a.row_of[static_cast<size_t>(t) * a.K + j];
         s_row[j] = (r >= 0 && r < A) ? r : 0;
-        s_w[j] = a.w[static_cast<size_t>(t) * a.K + j];
+        s_w[j] = j < a.k ? a.w[static_cast<size_t>(t) * a.k + j] : 1.0f;   // shared expert: weight 1
     }
     __syncthreads();
     const int c = blockIdx.y * blockDim.x + threadIdx.x;

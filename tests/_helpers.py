@@ -94,7 +94,7 @@ class GpuProblem:
         [A, kdim/g]: fp32 for recipe 0, UE8M0 bytes for recipe 1."""
         SR = self.layout["scale_rows"]
         nb = kdim // 128
-        A = self.shape.num_tokens * self.shape.top_k
+        A = self.shape.num_tokens * (self.shape.top_k + self.shape.shared_experts)
         words = self.ws_region(name, torch.int32, nb * SR).cpu().numpy().reshape(nb, SR)[:, :A]
         if self.shape.recipe == 0:
             return np.ascontiguousarray(words.view(np.float32).T)

@@ -28,7 +28,10 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_config_struct_layout():
-    assert ctypes.sizeof(moe._Cfg) == 48
+    # moe_config_t: twelve 4-byte fields in header order, shared_experts last
+    assert ctypes.sizeof(moe._Cfg) == 52
+    assert moe._Cfg.shared_experts.offset == 48
+    assert moe._Cfg.recipe.offset == 44
 
 
 def cfg(**kw):
@@ -51,6 +54,8 @@ def cfg(**kw):
     (dict(group_count=4, k_group=5), moe.MOE_ERR_UNSUPPORTED),
     (dict(group_count=4, k_group=1, top_k=3), moe.MOE_ERR_UNSUPPORTED),
     (dict(group_count=8, group_select_mode=1), moe.MOE_ERR_UNSUPPORTED),
+    (dict(shared_experts=2), moe.MOE_ERR_UNSUPPORTED),
+    (dict(shared_experts=-1), moe.MOE_ERR_UNSUPPORTED),
 ])
 def test_validation(kw, code):
     with pytest.raises(moe.MoeError) as e:
@@ -73,6 +78,27 @@ def test_valid_configs_and_sizes():
         w13, w13s, w2, w2s = moe.transformed_weights_size(c)
         assert w13 == s.num_experts * s.hidden * 2 * s.inter and w2 == s.num_experts * s.inter * s.hidden
         assert w13s == s.num_experts * (s.hidden // 128) * 2 * s.inter * 4
+
+
+def test_shared_expert_sizes():
+    """A shared expert adds one expert's weights and one row per token to the workspace."""
+    import synth
+    from dataclasses import replace
+    s = replace(synth.SHAPES["decode"], shared_experts=1)
+    c = moe.Config(**s.cfg())
+    moe.check_config(c)
+    c0 = moe.Config(**replace(s, shared_experts=0).cfg())
+    w = moe.transformed_weights_size(c)
+    w0 = moe.transformed_weights_size(c0)
+    E = s.num_experts
+    assert all(a * E == b * (E + 1) for a, b in zip(w, w0))
+    lay = moe.workspace_layout(c)
+    A = s.num_tokens * (s.top_k + 1)
+    assert lay["o"] + 4 * A * s.hidden <= lay["total"]
+    assert lay["scale_rows"] >= A
+    assert lay["total"] > moe.workspace_size(c0)
+    # 256 routed experts plus a shared one are accepted
+    moe.check_config(moe.Config(**replace(synth.SHAPES["prefill"], shared_experts=1).cfg()))
 
 
 def test_forward_rejects_bad_pointers_before_any_cuda_call():
