@@ -1,7 +1,7 @@
 """Benchmark of the fused FP8 routed-expert MoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|tiny|prefill|skewed|large]
-                    [--impl reference] [--no-cpu-baseline]
+                    [--impl reference] [--no-cpu-baseline] [--tokens T] [--shared-expert]
 
 One step = one moe_forward call (route, permute, quantize, gate+up GEMM with SwiGLU and
 requantization, down GEMM, combine) over one batch of seeded synthetic inputs of the named
@@ -68,6 +68,7 @@ def describe(shape: synth.Shape) -> str:
     rec = "E4M3 + fp32 scale per (row,128)" if shape.recipe == 0 else "MXFP8 (E4M3 + UE8M0 per 32)"
     return (f"{shape.name}: {shape.num_tokens} tok, H {shape.hidden}, I {shape.inter}, "
             f"E {shape.num_experts}, top-{shape.top_k}, {rt}" + (", " + ", ".join(extra) if extra else "")
+            + (" + 1 shared expert" if shape.shared_experts else "")
             + f"; {rec}")
 
 
@@ -92,7 +93,7 @@ def algorithmic_bytes(shape, active):
 def gemm1_bytes(shape, active):
     """Algorithmic bytes of one gate+up launch: active experts' W13 codes + scales, the
     quantized activations read, the requantized SwiGLU products written."""
-    H, I, T, k = shape.hidden, shape.inter, shape.num_tokens, shape.top_k
+    H, I, T, k = shape.hidden, shape.inter, shape.num_tokens, shape.top_k + shape.shared_experts
     A = T * k
     g = 128 if shape.recipe == 0 else 32
     sb = 4 if shape.recipe == 0 else 1
@@ -101,7 +102,7 @@ def gemm1_bytes(shape, active):
 
 
 def gemm2_bytes(shape, active):
-    H, I, T, k = shape.hidden, shape.inter, shape.num_tokens, shape.top_k
+    H, I, T, k = shape.hidden, shape.inter, shape.num_tokens, shape.top_k + shape.shared_experts
     A = T * k
     g = 128 if shape.recipe == 0 else 32
     sb = 4 if shape.recipe == 0 else 1
@@ -220,6 +221,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override the problem's token count (reduced cases for profiler captures)")
+    ap.add_argument("--shared-expert", action="store_true",
+                    help="add a shared expert (every token, weight 1) to the problem")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -229,6 +232,9 @@ def main():
     shape = synth.SHAPES[args.config]
     if args.tokens:
         shape = shape.with_tokens(args.tokens)
+    if args.shared_expert:
+        from dataclasses import replace
+        shape = replace(shape, shared_experts=1)
 
     if args.impl == "reference":
         reference_arm(args, shape, rank)
@@ -254,7 +260,7 @@ def main():
         del d.w13, d.w2
     ws = moe.new_workspace(cfg, dev)
     y = torch.empty((shape.num_tokens, shape.hidden), dtype=torch.bfloat16, device=dev)
-    counts = torch.zeros(shape.num_experts, dtype=torch.int32, device=dev)
+    counts = torch.zeros(shape.num_experts + shape.shared_experts, dtype=torch.int32, device=dev)
 
     def step(profile=None):
         moe.forward(cfg, d.x, weights, router_logits=d.logits, per_expert_scale=d.per_expert_scale,
@@ -266,7 +272,7 @@ def main():
     torch.cuda.synchronize()
     status = moe.read_status(ws)
     active = int((counts.cpu() > 0).sum())
-    A = shape.num_tokens * shape.top_k
+    A = shape.num_tokens * (shape.top_k + shape.shared_experts)   # rows through the GEMMs
 
     # timed region: K plain forwards (no events between the kernels, which would break their
     # programmatic-dependent-launch overlap)
@@ -356,7 +362,8 @@ def main():
         # the library's kernel choice: MXFP8 -> block-scaled kernel; fp32 scales -> swap-AB narrow
         # kernel at <= 32 routed rows per expert, else the wide kernel
         kname = ("k_grouped_gemm_mx" if shape.recipe == 1 else
-                 "k_grouped_gemm_narrow" if A <= 32 * shape.num_experts else "k_grouped_gemm")
+                 "k_grouped_gemm_narrow" if A <= 32 * (shape.num_experts + shape.shared_experts)
+                 else "k_grouped_gemm")
         roof.update({"kernel": kname + "<gate+up>",
                      "traffic": traffic_for("gemm1", shape.name),
                      "peak_source": f"{pk_kind} ({'sustained bf16 x2 for fp8' if compute_bound else 'copy'})",
