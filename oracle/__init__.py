@@ -110,6 +110,8 @@ def _load():
             lib.orc_check_cfg.argtypes = [ctypes.POINTER(_Cfg)]
             lib.orc_route.restype = ctypes.c_int
             lib.orc_route.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P]
+            lib.orc_gate_logits.restype = None
+            lib.orc_gate_logits.argtypes = [ctypes.c_int] * 3 + [P] * 3 + [ctypes.c_float, P]
             lib.orc_permute.restype = None
             lib.orc_permute.argtypes = [ctypes.c_int] * 3 + [P] * 5
             lib.orc_scaled_gemv.restype = None
@@ -239,6 +241,18 @@ def scaled_gemv(recipe: int, aq, as_, wq, ws):
     K, N = wq.shape
     out = np.zeros(N, np.float64)
     _load().orc_scaled_gemv(recipe, K, N, _p(aq), _p(as_), _p(wq), _p(ws), _p(out))
+    return out
+
+
+def gate_logits(x_bf16, norm_w, router_w, eps: float) -> np.ndarray:
+    """RMSNorm + router matmul (the gate in front of the router): fp32 logits [T, E]."""
+    x = _arr(x_bf16, np.uint16)
+    nw = _arr(norm_w, np.float32)
+    rw = _arr(router_w, np.float32)
+    T, H = x.shape
+    E = rw.shape[0]
+    out = np.zeros((T, E), np.float32)
+    _load().orc_gate_logits(T, H, E, _p(x), _p(nw), _p(rw), ctypes.c_float(eps), _p(out))
     return out
 
 

@@ -340,6 +340,37 @@ int orc_route(const orc_cfg *c, const float *logits, const float *per_expert_sca
 }
 
 /* ------------------------------------------------------------------------------------------
+ * The gate in front of the router ([mlx_native] moe_gate: RMS-Norm of the token's hidden state,
+ * then the router matmul, then top-K with softmax and per-expert scale), up to the logits:
+ *   xn[h]      = x[h] / sqrt( mean_h x[h]^2 + eps ) * norm_w[h]
+ *   logits[e]  = sum_h xn[h] * router_w[e, h]          (router_w fp32 [E, H], row-major)
+ * in fp64, rounded once to fp32 (the router takes fp32 logits).  Reading: the learned norm
+ * weight multiplies the normalized value (the page names it "RMS norm learned weight").
+ * ---------------------------------------------------------------------------------------- */
+void orc_gate_logits(int T, int H, int E, const uint16_t *x, const float *norm_w,
+                     const float *router_w, float eps, float *logits)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; t++) {
+        double ss = 0.0;
+        double *xn = (double *)malloc(sizeof(double) * (size_t)H);
+        for (int h = 0; h < H; h++) {
+            const double v = (double)bf16_to_f32(x[(size_t)t * H + h]);
+            ss += v * v;
+        }
+        const double r = 1.0 / sqrt(ss / (double)H + (double)eps);
+        for (int h = 0; h < H; h++)
+            xn[h] = (double)bf16_to_f32(x[(size_t)t * H + h]) * r * (double)norm_w[h];
+        for (int e = 0; e < E; e++) {
+            double acc = 0.0;
+            for (int h = 0; h < H; h++) acc += xn[h] * (double)router_w[(size_t)e * H + h];
+            logits[(size_t)t * E + e] = (float)acc;
+        }
+        free(xn);
+    }
+}
+
+/* ------------------------------------------------------------------------------------------
  * Permutation into expert-contiguous order ([MindIE] execution flow, dispatch: tokens are
  * reordered by expert and the tokens per expert counted; combine restores token order).
  * Routed row a = t*k + j.  Reading: inside one expert, rows ascend by token index.

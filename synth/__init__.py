@@ -34,7 +34,7 @@ import torch
 E4M3_MAX = 448.0
 
 # tensor ids folded into the seeds
-_X, _LOGITS, _BIAS_ROUTE, _PES, _W13, _W2, _B13, _B2, _RANK = range(9)
+_X, _LOGITS, _BIAS_ROUTE, _PES, _W13, _W2, _B13, _B2, _RANK, _NORM_W, _ROUTER_W = range(11)
 
 
 @dataclass(frozen=True)
@@ -198,6 +198,16 @@ def make_activations(shape: Shape, device="cpu", num_tokens: int | None = None):
     if shape.per_expert_scale:
         pes = torch.rand((E,), generator=_gen(device, shape.seed, _PES), device=device) + 0.5
     return x, logits.contiguous(), pes
+
+
+def make_gate(shape: Shape, device="cpu"):
+    """Inputs of the gate in front of the router: the RMSNorm weight fp32 [H] ~ 1 + N(0, 0.1),
+    the router weight fp32 [E, H] ~ N(0, 1/sqrt(H)) (so the logits are about N(0, 1)), and the
+    norm epsilon."""
+    H, E = shape.hidden, shape.num_experts
+    norm_w = 1.0 + _randn((H,), 0.1, device, shape.seed, _NORM_W)
+    router_w = _randn((E, H), 1.0 / math.sqrt(H), device, shape.seed, _ROUTER_W)
+    return norm_w.contiguous(), router_w.contiguous(), 1e-6
 
 
 def make_problem(name_or_shape, device="cpu", num_tokens: int | None = None) -> Problem:
