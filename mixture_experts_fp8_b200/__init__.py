@@ -35,7 +35,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_forward", "moe_forward_profiled",
     "moe_profile_create", "moe_profile_destroy", "moe_profile_read", "moe_profile_reset",
     "moe_read_status", "moe_selftest_bounded_wait", "moe_forward_static_workspace",
-    "moe_debug_inject_fault",
+    "moe_debug_inject_fault", "moe_gate",
 )
 MOE_FAULT_NONE = 0
 MOE_FAULT_SKIP_STAGE = 1
@@ -132,6 +132,7 @@ def _load():
             "moe_selftest_bounded_wait": [P, ctypes.c_uint32, P],
             "moe_forward_static_workspace": [CP] + [P] * 13 + [P],
             "moe_debug_inject_fault": [I],
+            "moe_gate": [CP, P, P, P, ctypes.c_float, P, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -219,6 +220,26 @@ def route(cfg: Config, router_logits, per_expert_scale=None, topk_idx=None, topk
     _check(_load().moe_route(ctypes.byref(c), _ptr(router_logits), _ptr(per_expert_scale),
                              _ptr(topk_idx), _ptr(topk_weights), _stream(stream)))
     return topk_idx, topk_weights
+
+
+def gate(cfg: Config, hidden_states, norm_weight, router_weight, rms_eps: float,
+         per_expert_scale=None, logits=None, topk_idx=None, topk_weights=None, stream=None):
+    """RMSNorm + router matmul + router top-k in one launch.
+    -> (logits fp32 [T, E], topk_idx int32 [T, k], topk_weights fp32 [T, k])."""
+    import torch
+    T, E, k = cfg.num_tokens, cfg.num_experts, cfg.top_k
+    dev = hidden_states.device
+    if logits is None:
+        logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    if topk_idx is None:
+        topk_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if topk_weights is None:
+        topk_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
+    c = cfg.c()
+    _check(_load().moe_gate(ctypes.byref(c), _ptr(hidden_states), _ptr(norm_weight), _ptr(router_weight),
+                            ctypes.c_float(rms_eps), _ptr(per_expert_scale), _ptr(logits), _ptr(topk_idx),
+                            _ptr(topk_weights), _stream(stream)))
+    return logits, topk_idx, topk_weights
 
 
 def forward(cfg: Config, hidden_states, weights, router_logits=None, per_expert_scale=None,

@@ -36,6 +36,15 @@ struct RouteArgs {
     int32_t* status;            // cleared to MOE_OK by the first thread when non-null
 };
 
+struct GateArgs {
+    const __nv_bfloat16* x;     // [T, H]
+    const float* norm_w;        // [H]
+    const float* router_w;      // [E, H]
+    float* logits;              // [T, E] out
+    float eps;
+    int T, H, E;
+};
+
 // Rows r = t * KT + j of the permutation: slot j < k is routed to idx[t * k + j]; slot k (when
 // KT > k) is the shared expert, index E, which every token uses.
 struct PermuteArgs {
@@ -101,6 +110,8 @@ struct GemmArgs {
 };
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+cudaError_t launch_gate(const GateArgs& g, const RouteArgs& ra, cudaStream_t s);
+size_t gate_smem_bytes(int H);
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 cudaError_t launch_permute_small(const PermuteArgs& pa, bool clear_status, cudaStream_t s);
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s);

@@ -420,6 +420,30 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     return ok();
 }
 
+int moe_gate(const moe_config_t* cfg, const void* hidden_states, const float* norm_weight,
+             const float* router_weight, float rms_eps, const float* per_expert_scale, float* logits,
+             int32_t* topk_idx, float* topk_weights, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!hidden_states || !norm_weight || !router_weight || !logits || !topk_idx || !topk_weights)
+        return fail(MOE_ERR_INVALID_ARG, "moe_gate: NULL pointer");
+    if (!aligned(hidden_states, 16) || !aligned(router_weight, 16) || !aligned(norm_weight, 4) ||
+        !aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_weights, 4) ||
+        (per_expert_scale && !aligned(per_expert_scale, 4)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_gate: misaligned buffer (hidden_states and router_weight need 16 bytes)");
+    if (!(rms_eps >= 0.0f)) return fail(MOE_ERR_INVALID_ARG, "moe_gate: rms_eps must be >= 0");
+    if (cfg->hidden > 12288) return fail(MOE_ERR_UNSUPPORTED, "moe_gate: hidden (%d) exceeds 12288", cfg->hidden);
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    moe::GateArgs g{static_cast<const __nv_bfloat16*>(hidden_states), norm_weight, router_weight, logits, rms_eps,
+                    cfg->num_tokens, cfg->hidden, cfg->num_experts};
+    moe::RouteArgs ra{logits, per_expert_scale, topk_idx, topk_weights, cfg->num_tokens, cfg->num_experts,
+                      cfg->top_k, cfg->routing, cfg->renormalize, cfg->group_count, cfg->k_group,
+                      cfg->group_select_mode, cfg->routed_scaling_factor, nullptr};
+    MOE_CUDA_TRY(moe::launch_gate(g, ra, static_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
 int moe_forward(const moe_config_t* cfg, const void* hidden_states, const float* router_logits,
                 const float* per_expert_scale, const int32_t* topk_idx, const float* topk_weights, const void* w13_t,
                 const void* w13s_t, const void* w2_t, const void* w2s_t, const void* w13_bias, const void* w2_bias,

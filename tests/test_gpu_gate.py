@@ -1,0 +1,96 @@
+"""Parity of the fused gate (RMSNorm + router matmul + router top-k, "mlx_native
+ops/moe_gate.rs") against the oracle: logits within fp32-vs-fp64 accumulation error, the top-k
+bit-exact against the oracle's router run on the GPU's own logits, and against the oracle's gate
+except where two candidate logits lie within that error; logits independent of the batch; the
+gate's routing feeds the layer exactly as router logits do."""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from _helpers import GpuProblem, bits, check_routing, oracle_cfg
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "decode": synth.SHAPES["decode"],                                         # softmax, per-expert scale
+    "prefill64": synth.SHAPES["prefill"].with_tokens(64),                     # sigmoid, groups, H 7168
+    "small": synth.Shape("gsmall", 37, 384, 128, 24, 3, renormalize=1, seed=42),
+}
+LOGIT_TOL = 3e-5          # |gpu - oracle| relative to max |logit|: fp32 sums over H terms
+
+
+class _Acts:
+    """The gate's inputs only (no expert weights): x, per-expert scale, and their numpy view."""
+
+    def __init__(self, shape):
+        self.x, _, self.per_expert_scale = synth.make_activations(shape)
+
+    def numpy_inputs(self):
+        return dict(x=self.x.view(torch.int16).numpy().view(np.uint16), logits=None,
+                    per_expert_scale=None if self.per_expert_scale is None else self.per_expert_scale.numpy())
+
+
+def _gate_inputs(shape, full=False):
+    prob = synth.make_problem(shape) if full else _Acts(shape)
+    nw, rw, eps = synth.make_gate(shape)
+    return prob, nw, rw, eps
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_gate_logits_and_routing(name):
+    import mixture_experts_fp8_b200 as moe
+    shape = CASES[name]
+    prob, nw, rw, eps = _gate_inputs(shape)
+    ni = prob.numpy_inputs()
+    cfg = moe.Config(**shape.cfg())
+    x = prob.x.cuda()
+    pes = None if prob.per_expert_scale is None else prob.per_expert_scale.cuda()
+    lg, idx, w = moe.gate(cfg, x, nw.cuda(), rw.cuda(), eps, per_expert_scale=pes)
+    torch.cuda.synchronize()
+    lg = lg.cpu().numpy()
+    ref = oracle.gate_logits(ni["x"], nw.numpy(), rw.numpy(), eps)
+    err = np.max(np.abs(lg - ref)) / np.max(np.abs(ref))
+    assert err <= LOGIT_TOL, err
+    # the router on the GPU's own logits: exactly the oracle's router on them
+    gni = dict(ni, logits=lg)
+    check_routing(shape, gni, idx.cpu().numpy(), w.cpu().numpy())
+    # against the oracle's gate: equal except where the k-th and (k+1)-th choices are closer
+    # than the logit error
+    ridx, _, tie = oracle.route(oracle_cfg(shape), ref, ni["per_expert_scale"])
+    gidx = idx.cpu().numpy()
+    diff = np.where(np.any(ridx != gidx, axis=1))[0]
+    for t in diff:
+        s = np.sort(ref[t])[::-1]
+        close = np.min(np.abs(np.diff(s))) <= 4 * LOGIT_TOL * np.max(np.abs(ref))
+        assert close or tie[t], f"token {t}: routing differs without a near tie"
+    assert diff.size <= max(1, shape.num_tokens // 50)
+
+
+def test_gate_logits_do_not_depend_on_the_batch():
+    import mixture_experts_fp8_b200 as moe
+    shape = CASES["small"]
+    prob, nw, rw, eps = _gate_inputs(shape)
+    cfg = moe.Config(**shape.cfg())
+    x = prob.x.cuda()
+    lg, _, _ = moe.gate(cfg, x, nw.cuda(), rw.cuda(), eps)
+    sel = torch.tensor([36, 0, 5, 5, 17], device="cuda")
+    cs = moe.Config(**replace(shape, num_tokens=5).cfg())
+    ls, _, _ = moe.gate(cs, x[sel].contiguous(), nw.cuda(), rw.cuda(), eps)
+    torch.cuda.synchronize()
+    assert torch.equal(ls, lg[sel])
+
+
+def test_gate_routing_drives_the_layer_like_router_logits():
+    import mixture_experts_fp8_b200 as moe
+    shape = CASES["decode"]
+    prob, nw, rw, eps = _gate_inputs(shape, full=True)
+    gp = GpuProblem(prob)
+    lg, idx, w = moe.gate(gp.cfg, gp.d.x, nw.cuda(), rw.cuda(), eps, per_expert_scale=gp.d.per_expert_scale)
+    y1 = bits(gp.forward(topk_idx=idx, topk_weights=w))
+    y2 = bits(gp.forward(logits=lg))
+    assert gp.status() == 0
+    assert np.array_equal(y1, y2)
