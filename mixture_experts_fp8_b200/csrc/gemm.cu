@@ -366,16 +366,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int h = 0; h < 2; ++h) {
                         const int c0 = nb * kTileN + h * kHalf + qtr * 32;
                         if (c0 < p.N) {
-                            float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.N + c0);
+                            float* dst = p.out + static_cast<size_t>(r) * p.N + c0;
                             const uint4* b4 =
                                 p.bias ? reinterpret_cast<const uint4*>(p.bias + static_cast<size_t>(e) * p.N + c0)
                                        : nullptr;
 #pragma unroll
-                            for (int c = 0; c < 32; c += 8) {   // 8 columns: one bias load, two stores
+                            for (int c = 0; c < 32; c += 8) {   // 8 columns: one bias load, one 32-byte store
                                 float* a = acc + 32 * h + c;
                                 if (b4) add_bias8(a, ld_nc_u4(b4 + (c >> 3)));
-                                dst[c >> 2] = make_float4(a[0], a[1], a[2], a[3]);
-                                dst[(c >> 2) + 1] = make_float4(a[4], a[5], a[6], a[7]);
+                                st_global_f32x8(dst + c, a);
                             }
                         }
                     }

@@ -313,9 +313,9 @@ __global__ void __launch_bounds__(kXThreads, 1)
                     add_bias32(acc, p.bias + static_cast<size_t>(e) * p.N + c0);
                     add_bias32(acc + 32, p.bias + static_cast<size_t>(e) * p.N + c0 + 32);
                 }
-                float4* dst = reinterpret_cast<float4*>(p.out + static_cast<size_t>(r) * p.N + c0);
+                float* dst = p.out + static_cast<size_t>(r) * p.N + c0;
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) dst[c >> 2] = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
+                for (int c = 0; c < 64; c += 8) st_global_f32x8(dst + c, acc + c);
             }
         }
     }
