@@ -66,7 +66,8 @@ class Config:
     k_group: int = 1
     group_select_mode: int = 0
     routed_scaling_factor: float = 1.0
-    recipe: int = 0              # 0 fp32 scale per (row,128); 1 UE8M0 per 32
+    recipe: int = 0              # 0 fp32 scale per (row,128); 1 UE8M0 per 32 (MXFP8);
+                                 # 2 W4A8: E2M1 weights (two per byte) + UE8M0 per 32, MXFP8 acts
     shared_experts: int = 0      # 1: one more expert (index num_experts), every token, weight 1
 
     @property
@@ -98,6 +99,8 @@ def _load():
             P = ctypes.c_void_p
             lib.orc_e4m3_decode.restype = ctypes.c_double
             lib.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.orc_e2m1_decode.restype = ctypes.c_double
+            lib.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
             lib.orc_e4m3_encode.restype = ctypes.c_uint8
             lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
             lib.orc_mx_exponent.restype = ctypes.c_int
@@ -143,6 +146,10 @@ def _arr(a, dtype):
 # ----------------------------------------------------------------------------- scalar pieces
 def e4m3_decode(code: int) -> float:
     return _load().orc_e4m3_decode(int(code) & 0xFF)
+
+
+def e2m1_decode(code: int) -> float:
+    return float(_load().orc_e2m1_decode(code))
 
 
 def e4m3_encode(v: float) -> int:
@@ -232,13 +239,14 @@ def permute(topk_idx: np.ndarray, num_experts: int):
 
 
 def scaled_gemv(recipe: int, aq, as_, wq, ws):
-    """One block-scaled FP8 GEMM row: aq [K] codes, as_ [K/g], wq [K,N] codes, ws [K/g,N]."""
+    """One block-scaled GEMM row: aq [K] E4M3 codes, as_ [K/g], wq [K,N] codes (recipe 2:
+    [K,N/2] bytes of two E2M1 codes, the even column in the low nibble), ws [K/g,N]."""
     aq = _arr(aq, np.uint8).ravel()
     wq = _arr(wq, np.uint8)
     sd = np.float32 if recipe == 0 else np.uint8
     as_ = _arr(as_, sd).ravel()
     ws = _arr(ws, sd)
-    K, N = wq.shape
+    K, N = wq.shape[0], wq.shape[1] * (2 if recipe == 2 else 1)
     out = np.zeros(N, np.float64)
     _load().orc_scaled_gemv(recipe, K, N, _p(aq), _p(as_), _p(wq), _p(ws), _p(out))
     return out

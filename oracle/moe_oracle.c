@@ -18,6 +18,9 @@
  *              4-packed scale factors, per-32 activation scale factors), Testing.
  *   [mlx]      "mlx_native ops/moe_gate.rs": moe_gate doc (top-K sort, softmax,
  *              per_expert_scale) and its argument validation.
+ *   [W4A8]     "DeepGEMM PR #371", Changes: the W4A8 (FP8 x FP4) path it derives from uses
+ *              e2m1 weights with the same 4-packed UE8M0 scale factors; "MATE Mega MoE",
+ *              Use Mega MoE when: the W4A8 mixed-dtype GEMM path.
  *
  * Precision: decisions that turn floating point into integers (expert selection, group
  * selection, E4M3 codes, scales) are taken in fp32, the precision of the kernels; every
@@ -47,7 +50,8 @@ typedef struct {
     int32_t renormalize;        /* softmax only; sigmoid weights are always normalized       */
     int32_t group_count, k_group, group_select_mode;
     float routed_scaling_factor;
-    int32_t recipe;             /* 0: fp32 scale per (row,128); 1: UE8M0 scale per 32 (MXFP8) */
+    int32_t recipe;             /* 0: fp32 scale per (row,128); 1: UE8M0 scale per 32 (MXFP8);
+                                   2: W4A8, E2M1 weights with UE8M0 per 32, MXFP8 activations */
     int32_t shared_experts;     /* 0 or 1: one more expert, index num_experts, that every token
                                    uses with weight 1 ([metrale] run_fp8_grouped_w8a8: the shared
                                    expert's gate/up/down run in the same grouped steps)          */
@@ -106,6 +110,36 @@ __attribute__((constructor)) static void fill_e4m3_table(void)
     for (int c = 0; c < 256; c++) e4m3_table[c] = orc_e4m3_decode((uint8_t)c);
 }
 
+/* ------------------------------------------------------------------------------------------
+ * E2M1 (FP4, the "e2m1" weights of [W4A8]; the element format of the OCP microscaling
+ * formats): 1 sign, 2 exponent (bias 1), 1 mantissa bit; no infinities or NaN.  Exponent 0 is
+ * subnormal, m * 0.5; otherwise (1 + m/2) * 2^(e-1).  Magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+ * Reading: two codes per byte, the lower-indexed element in the low nibble.
+ * ---------------------------------------------------------------------------------------- */
+double orc_e2m1_decode(uint8_t c)
+{
+    int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+    double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -v : v;
+}
+
+/* Weight element n of row k of a [Kdim, N] weight matrix: an E4M3 byte (recipes 0, 1) or an
+ * E2M1 nibble of a byte packed along N (recipe 2). */
+static double weight_value(int recipe, const uint8_t *wq, int N, int k, int n)
+{
+    if (recipe == 2) {
+        const uint8_t b = wq[(size_t)k * (N / 2) + n / 2];
+        return orc_e2m1_decode((uint8_t)((n & 1) ? (b >> 4) : (b & 15)));
+    }
+    return e4m3_table[wq[(size_t)k * N + n]];
+}
+
+/* Bytes of a [Kdim, N] weight matrix's codes. */
+static size_t weight_bytes(int recipe, int Kdim, int N)
+{
+    return recipe == 2 ? (size_t)Kdim * N / 2 : (size_t)Kdim * N;
+}
+
 /* UE8M0: an unsigned biased power-of-two exponent, value 2^(b - 127). */
 static double ue8m0_value(uint8_t b) { return ldexp(1.0, (int)b - 127); }
 
@@ -152,8 +186,9 @@ void orc_quant_group_mx(const float *x, int n, uint8_t *q, uint8_t *e8_out)
     *e8_out = (uint8_t)(e + 127);
 }
 
-/* Quantize one row of n values in groups: recipe 0 -> n/128 fp32 scales, recipe 1 -> n/32
- * UE8M0 bytes.  `scales` points at float or uint8_t storage accordingly. */
+/* Quantize one row of n values in groups: recipe 0 -> n/128 fp32 scales, recipes 1 and 2
+ * (W4A8 activations are MXFP8) -> n/32 UE8M0 bytes.  `scales` points at float or uint8_t
+ * storage accordingly. */
 void orc_quant_row(const float *x, int n, int recipe, uint8_t *q, void *scales)
 {
     if (recipe == 0) {
@@ -231,7 +266,7 @@ int orc_check_cfg(const orc_cfg *c)
     if (c->top_k > c->k_group * (c->num_experts / c->group_count)) return ORC_EUNSUPPORTED;
     if (c->group_select_mode == 1 && c->num_experts / c->group_count < 2) return ORC_EUNSUPPORTED;
     if (c->routing != 0 && c->routing != 1) return ORC_EINVAL;
-    if (c->recipe != 0 && c->recipe != 1) return ORC_EINVAL;
+    if (c->recipe < 0 || c->recipe > 2) return ORC_EINVAL;
     if (c->shared_experts != 0 && c->shared_experts != 1) return ORC_EUNSUPPORTED;
     return ORC_OK;
 }
@@ -396,6 +431,7 @@ void orc_permute(int T, int K, int E, const int32_t *topk_idx, int32_t *counts,
 /* ------------------------------------------------------------------------------------------
  * One grouped, block-scaled FP8 GEMM row:
  *   out[n] = sum_g  sa[g] * sw[g][n] * sum_{k in group g} dec(aq[k]) * dec(wq[k][n])
+ * (dec = E4M3, or E2M1 for the W4A8 weights of recipe 2, which are packed two per byte along N)
  * with wq stored K rows x N columns (the pages' w13 [E, hidden, 2*inter] and
  * w2 [E, inter, hidden] orientation, [MindIE] parameter table) and the weight scales stored
  * [K/g][N] ([MindIE] MXFP8 example: the scale tensor is transposed to put the K blocks
@@ -417,8 +453,7 @@ void orc_scaled_gemv(int recipe, int Kdim, int N, const uint8_t *aq, const void 
         for (int n = 0; n < N; n++) part[n] = 0.0;
         for (int k = grp * g; k < (grp + 1) * g; k++) {
             double a = e4m3_table[aq[k]];
-            const uint8_t *wrow = wq + (size_t)k * N;
-            for (int n = 0; n < N; n++) part[n] += a * e4m3_table[wrow[n]];
+            for (int n = 0; n < N; n++) part[n] += a * weight_value(recipe, wq, N, k, n);
         }
         for (int n = 0; n < N; n++)
             out[n] += sa * act_scale(recipe, ws, (size_t)grp * N + n) * part[n];
@@ -435,8 +470,10 @@ void orc_scaled_gemv(int recipe, int Kdim, int N, const uint8_t *aq, const void 
  *   o    = gemm(a_q, W2_e) + b2_e                             (H values, fp64)
  * ---------------------------------------------------------------------------------------- */
 typedef struct {
-    const uint8_t *w13;   const void *w13s;   /* [E,H,2I] codes, scales [E,H/g,2I]   */
-    const uint8_t *w2;    const void *w2s;    /* [E,I,H] codes,  scales [E,I/g,H]    */
+    const uint8_t *w13;   const void *w13s;   /* [E,H,2I] codes (recipe 2: [E,H,I] bytes of
+                                                 two E2M1 codes), scales [E,H/g,2I]      */
+    const uint8_t *w2;    const void *w2s;    /* [E,I,H] codes (recipe 2: [E,I,H/2]), scales
+                                                 [E,I/g,H]                               */
     const uint16_t *b13;  const uint16_t *b2; /* bf16 [E,2I], [E,H], or NULL         */
 } orc_weights;
 
@@ -452,7 +489,7 @@ static void expert_mlp_row(const orc_cfg *c, const orc_weights *W, int e, const 
     uint8_t *aq = (uint8_t *)malloc((size_t)I);
     void *as = malloc(sb * (size_t)(I / g));
 
-    orc_scaled_gemv(c->recipe, H, 2 * I, xq, xs, W->w13 + (size_t)e * H * 2 * I,
+    orc_scaled_gemv(c->recipe, H, 2 * I, xq, xs, W->w13 + (size_t)e * weight_bytes(c->recipe, H, 2 * I),
                     (const uint8_t *)W->w13s + (size_t)e * (H / g) * 2 * I * sb, h);
     if (W->b13)
         for (int n = 0; n < 2 * I; n++) h[n] += (double)bf16_to_f32(W->b13[(size_t)e * 2 * I + n]);
@@ -461,7 +498,7 @@ static void expert_mlp_row(const orc_cfg *c, const orc_weights *W, int e, const 
         a[i] = (float)(z / (1.0 + exp(-z)) * h[I + i]);
     }
     orc_quant_row(a, I, c->recipe, aq, as);
-    orc_scaled_gemv(c->recipe, I, H, aq, as, W->w2 + (size_t)e * I * H,
+    orc_scaled_gemv(c->recipe, I, H, aq, as, W->w2 + (size_t)e * weight_bytes(c->recipe, I, H),
                     (const uint8_t *)W->w2s + (size_t)e * (I / g) * H * sb, o);
     if (W->b2)
         for (int n = 0; n < H; n++) o[n] += (double)bf16_to_f32(W->b2[(size_t)e * H + n]);

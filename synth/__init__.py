@@ -21,6 +21,8 @@ Shapes and distributions (one line per problem):
           ln p_e with p_e ~ rank(e)^-1.2 (Zipf, rank a seeded permutation); MXFP8, seed 3
   large   16384 tok, H 4096, I 1536, E 128, k 8, softmax + renormalize; biases bf16
           N(0,0.02), seed 4
+  decode_w4a8 / prefill_w4a8: the decode and prefill shapes with W4A8 weights (E2M1 codes,
+          UE8M0 per 32, nearest-even rounding) and MXFP8 activations, seeds 5 and 6
   x ~ N(0,1) rounded to bf16; logits fp32; weights N(0, 1/sqrt(K)) with K the contraction dim.
 """
 from __future__ import annotations
@@ -51,7 +53,8 @@ class Shape:
     k_group: int = 1
     group_select_mode: int = 0
     routed_scaling_factor: float = 1.0
-    recipe: int = 0                  # 0 fp32 per (row,128); 1 MXFP8 (UE8M0 per 32)
+    recipe: int = 0                  # 0 fp32 per (row,128); 1 MXFP8 (UE8M0 per 32);
+                                     # 2 W4A8: E2M1 weights + UE8M0 per 32, MXFP8 activations
     seed: int = 0
     logit_bias_std: float = 0.0      # per-expert bias added to the logits
     zipf_s: float = 0.0              # > 0: add ln p_e, p_e ~ rank^-s
@@ -87,6 +90,12 @@ SHAPES = {
                     seed=3, zipf_s=1.2),
     "large": Shape("large", 16384, 4096, 1536, 128, 8, routing=0, renormalize=1, seed=4,
                    biases=True),
+    # W4A8 (E2M1 weights, UE8M0 per 32; MXFP8 activations) on the decode and prefill shapes
+    "decode_w4a8": Shape("decode_w4a8", 64, 2816, 768, 128, 8, routing=0, renormalize=1,
+                         recipe=2, seed=5, per_expert_scale=True),
+    "prefill_w4a8": Shape("prefill_w4a8", 4096, 7168, 2048, 256, 8, routing=1, renormalize=1,
+                          group_count=8, k_group=4, group_select_mode=1,
+                          routed_scaling_factor=2.5, recipe=2, seed=6, logit_bias_std=0.1),
 }
 
 
@@ -109,14 +118,39 @@ def bf16_bits(t: torch.Tensor) -> torch.Tensor:
     return t.contiguous().view(torch.int16)
 
 
+E2M1_MAX = 6.0
+_E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)     # magnitudes of codes 0..7
+
+
+def _e2m1_codes(v: torch.Tensor) -> torch.Tensor:
+    """Nearest E2M1 code of each value (ties to the even code, saturating at 6): the input
+    recipe for the FP4 weights.  Returns uint8 codes 0..15 (bit 3 = sign)."""
+    grid = torch.tensor(_E2M1_GRID, dtype=torch.float32, device=v.device)
+    a = v.abs().clamp(max=E2M1_MAX)
+    lo = (torch.bucketize(a, grid, right=True) - 1).clamp(0, 7)
+    hi = (lo + 1).clamp(max=7)
+    dlo, dhi = a - grid[lo], grid[hi] - a
+    up = (dhi < dlo) | ((dhi == dlo) & (lo % 2 == 1))
+    code = torch.where(up, hi, lo)
+    return (code | ((v < 0) & (code > 0)).to(code.dtype) * 8).to(torch.uint8)
+
+
 def quantize_weight_block(w: torch.Tensor, recipe: int):
-    """Prepare one expert's weight w [K, N] (fp32) as E4M3 codes [K, N] (uint8) plus block
-    scales [K/g, N]: fp32 amax/448 per 128-deep block (recipe 0) or a UE8M0 power of two per
-    32-deep block (recipe 1).  Input preparation only; the cast is torch's."""
+    """Prepare one expert's weight w [K, N] (fp32) as codes plus block scales [K/g, N]: E4M3
+    codes [K, N] with fp32 amax/448 per 128-deep block (recipe 0) or a UE8M0 power of two per
+    32-deep block (recipe 1), or E2M1 codes packed two per byte along N, [K, N/2] (the even
+    column in the low nibble), with a UE8M0 power of two per 32-deep block, the smallest with
+    amax <= 6 * 2^e (recipe 2, the W4A8 weights).  Input preparation only; the E4M3 cast is
+    torch's."""
     K, N = w.shape
     g = 128 if recipe == 0 else 32
     blocks = w.reshape(K // g, g, N)
     amax = blocks.abs().amax(dim=1)                                   # [K/g, N]
+    if recipe == 2:
+        e = torch.ceil(torch.log2(torch.clamp(amax, min=1e-30) / E2M1_MAX)).clamp(-127, 127)
+        codes = _e2m1_codes((blocks / torch.exp2(e)[:, None, :]).reshape(K, N))
+        packed = codes[:, 0::2] | (codes[:, 1::2] << 4)
+        return packed.contiguous(), (e + 127).to(torch.uint8)
     if recipe == 0:
         scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
         sc_store = scale
@@ -135,9 +169,9 @@ class Problem:
     x: torch.Tensor                      # bf16 [T,H]
     logits: torch.Tensor                 # fp32 [T,E]
     per_expert_scale: torch.Tensor | None
-    w13: torch.Tensor                    # uint8 [E,H,2I]  (E + 1 experts with a shared expert)
+    w13: torch.Tensor                    # uint8 [E,H,2I] (W4A8: [E,H,I], two E2M1 codes a byte)
     w13_scale: torch.Tensor              # fp32 [E,H/128,2I] | uint8 [E,H/32,2I]
-    w2: torch.Tensor                     # uint8 [E,I,H]
+    w2: torch.Tensor                     # uint8 [E,I,H]  (W4A8: [E,I,H/2])
     w2_scale: torch.Tensor               # fp32 [E,I/128,H]  | uint8 [E,I/32,H]
     w13_bias: torch.Tensor | None        # bf16 [E,2I]
     w2_bias: torch.Tensor | None         # bf16 [E,H]
@@ -171,9 +205,10 @@ def make_weights(shape: Shape, device="cpu"):
     E, H, I, r = shape.num_experts + shape.shared_experts, shape.hidden, shape.inter, shape.recipe
     g = shape.group
     sdt = torch.float32 if r == 0 else torch.uint8
-    w13 = torch.empty((E, H, 2 * I), dtype=torch.uint8, device=device)
+    pk = 2 if r == 2 else 1                                  # E2M1 codes: two per byte
+    w13 = torch.empty((E, H, 2 * I // pk), dtype=torch.uint8, device=device)
     w13s = torch.empty((E, H // g, 2 * I), dtype=sdt, device=device)
-    w2 = torch.empty((E, I, H), dtype=torch.uint8, device=device)
+    w2 = torch.empty((E, I, H // pk), dtype=torch.uint8, device=device)
     w2s = torch.empty((E, I // g, H), dtype=sdt, device=device)
     for e in range(E):
         c, s = quantize_weight_block(_randn((H, 2 * I), 1.0 / math.sqrt(H), device, shape.seed, _W13, e), r)
