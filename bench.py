@@ -65,7 +65,8 @@ def describe(shape: synth.Shape) -> str:
         extra.append(f"rsf {shape.routed_scaling_factor}")
     if shape.biases:
         extra.append("biases")
-    rec = "E4M3 + fp32 scale per (row,128)" if shape.recipe == 0 else "MXFP8 (E4M3 + UE8M0 per 32)"
+    rec = {0: "E4M3 + fp32 scale per (row,128)", 1: "MXFP8 (E4M3 + UE8M0 per 32)",
+           2: "W4A8 (E2M1 weights + UE8M0 per 32, MXFP8 activations)"}[shape.recipe]
     return (f"{shape.name}: {shape.num_tokens} tok, H {shape.hidden}, I {shape.inter}, "
             f"E {shape.num_experts}, top-{shape.top_k}, {rt}" + (", " + ", ".join(extra) if extra else "")
             + (" + 1 shared expert" if shape.shared_experts else "")
@@ -80,11 +81,17 @@ def scale_bytes(shape, K, N):
     return (K // 128) * N * 4 if shape.recipe == 0 else (K // 32) * N
 
 
+def code_bytes(shape, K, N):
+    """Bytes of a [K, N] weight matrix's codes: one E4M3 byte each, or two E2M1 codes a byte."""
+    return K * N // 2 if shape.recipe == 2 else K * N
+
+
 def algorithmic_bytes(shape, active):
     """Minimum HBM bytes of one forward: each active expert's weights and scales once, plus the
     per-call tensors (x, y, logits).  Intermediates excluded."""
     H, I, E, T = shape.hidden, shape.inter, shape.num_experts, shape.num_tokens
-    w = active * (3 * H * I + scale_bytes(shape, H, 2 * I) + scale_bytes(shape, I, H))
+    w = active * (code_bytes(shape, H, 2 * I) + code_bytes(shape, I, H) + scale_bytes(shape, H, 2 * I)
+                  + scale_bytes(shape, I, H))
     if shape.biases:
         w += active * 2 * (2 * I + H)
     return w + 2 * T * H * 2 + 4 * T * E
@@ -97,7 +104,7 @@ def gemm1_bytes(shape, active):
     A = T * k
     g = 128 if shape.recipe == 0 else 32
     sb = 4 if shape.recipe == 0 else 1
-    return (active * (2 * I * H + scale_bytes(shape, H, 2 * I)) + A * H + A * (H // g) * sb
+    return (active * (code_bytes(shape, H, 2 * I) + scale_bytes(shape, H, 2 * I)) + A * H + A * (H // g) * sb
             + A * I + A * (I // g) * sb)
 
 
@@ -106,7 +113,7 @@ def gemm2_bytes(shape, active):
     A = T * k
     g = 128 if shape.recipe == 0 else 32
     sb = 4 if shape.recipe == 0 else 1
-    return active * (I * H + scale_bytes(shape, I, H)) + A * I + A * (I // g) * sb + A * H * 4
+    return active * (code_bytes(shape, I, H) + scale_bytes(shape, I, H)) + A * I + A * (I // g) * sb + A * H * 4
 
 
 class ClockSampler:
@@ -251,12 +258,13 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     dev = f"cuda:{local}"
-    gen_dev = dev if shape.name in ("prefill", "large") else "cpu"
+    big = shape.name in ("prefill", "large", "prefill_w4a8")     # inputs drawn on the device
+    gen_dev = dev if big else "cpu"
     prob = synth.make_problem(shape, device=gen_dev)
     d = prob.to(dev)
     cfg = moe.Config(**shape.cfg())
     weights = moe.transform_weights(cfg, d.w13, d.w13_scale, d.w2, d.w2_scale)
-    if shape.name in ("prefill", "large"):
+    if big:
         del d.w13, d.w2
     ws = moe.new_workspace(cfg, dev)
     y = torch.empty((shape.num_tokens, shape.hidden), dtype=torch.bfloat16, device=dev)
@@ -361,7 +369,7 @@ def main():
             roof = {"bound": "hbm", "achieved": g1_gbs, "peak": hbm, "unit": "GB/s", "frac": g1_gbs / hbm}
         # the library's kernel choice: MXFP8 -> block-scaled kernel; fp32 scales -> swap-AB narrow
         # kernel at <= 32 routed rows per expert, else the wide kernel
-        kname = ("k_grouped_gemm_mx" if shape.recipe == 1 else
+        kname = ("k_grouped_gemm_mx" if shape.recipe != 0 else
                  "k_grouped_gemm_narrow" if A <= 32 * (shape.num_experts + shape.shared_experts)
                  else "k_grouped_gemm")
         roof.update({"kernel": kname + "<gate+up>",

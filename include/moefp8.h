@@ -61,6 +61,12 @@ extern "C" {
  *   recipe             0 = E4M3 with an fp32 scale per (row, 128-element block) for
  *                          activations and per (output column, 128-deep K block) for weights
  *                      1 = MXFP8: E4M3 with a UE8M0 power-of-two scale per 32 elements
+ *                      2 = W4A8: weights E2M1 (FP4) with a UE8M0 scale per 32 K-elements,
+ *                          activations MXFP8 as recipe 1 ("DeepGEMM PR #371", Changes: the W4A8
+ *                          (FP8 x FP4) path, e2m1 weights with the same 4-packed UE8M0 scale
+ *                          factors; "MATE Mega MoE": the W4A8 mixed-dtype GEMM path).  Weight
+ *                          codes are packed two per byte along the last (N) dimension, the
+ *                          even column in the low nibble: w13 [E, H, I] and w2 [E, I, H/2] bytes.
  *   shared_experts     0, or 1: one more expert, index num_experts, that every token uses with
  *                      weight 1 after its top_k routed experts ("metrale_model_layers
  *                      fp8_grouped_tc_w8a8.rs", run_fp8_grouped_w8a8: the shared expert's
@@ -87,7 +93,7 @@ typedef struct {
  * expert), E' = num_experts + S, A = num_tokens * k' rows.  Scales are stored K-block-major: one 4-byte word per
  * (128-column block, row) with a row stride of scale_rows words; the word is the fp32 scale
  * (recipe 0) or the four UE8M0 bytes of the block's four 32-column groups, lowest group in the
- * lowest byte (recipe 1).  All offsets are multiples of 1024. */
+ * lowest byte (recipes 1 and 2).  All offsets are multiples of 1024. */
 typedef struct {
     size_t status;       /* int32 status word (MOE_OK or a device MOE_ERR_*)             */
     size_t topk_idx;     /* int32 [T, k]   routing computed by moe_forward               */
@@ -127,14 +133,16 @@ int moe_transformed_weights_size(const moe_config_t *cfg, size_t *w13_bytes, siz
 /* Re-lay the grouped FP8 expert weights for the forward ("MATE Mega MoE", Typical Flow step 2
  * and transform_weights_for_mega_moe).  Runs once, offline; deterministic and re-runnable.
  * (E below is num_experts + shared_experts: the shared expert's tensors come last.)
- *   w13        device, E4M3 codes [E, H, 2I] (K rows x N columns; columns 0:I gate, I:2I up)
- *   w13_scale  device, recipe 0: fp32 [E, H/128, 2I]; recipe 1: UE8M0 bytes [E, H/32, 2I]
- *   w2         device, E4M3 codes [E, I, H]
- *   w2_scale   device, recipe 0: fp32 [E, I/128, H];  recipe 1: UE8M0 bytes [E, I/32, H]
+ *   w13        device, E4M3 codes [E, H, 2I] (K rows x N columns; columns 0:I gate, I:2I up);
+ *              recipe 2: E2M1 codes two per byte along N, [E, H, I] bytes
+ *   w13_scale  device, recipe 0: fp32 [E, H/128, 2I]; recipes 1, 2: UE8M0 bytes [E, H/32, 2I]
+ *   w2         device, E4M3 codes [E, I, H]; recipe 2: [E, I, H/2] bytes of E2M1 pairs
+ *   w2_scale   device, recipe 0: fp32 [E, I/128, H];  recipes 1, 2: UE8M0 bytes [E, I/32, H]
  * (scales are K-block-major, the orientation of the "MindIE-SD Fused MoE" MXFP8 example.)
  * Outputs (device, sizes from moe_transformed_weights_size; opaque to the caller): K-major
- * codes with gate/up columns interleaved in 32-column blocks, and the scales re-laid to match.
- * Inputs and outputs must not overlap. */
+ * codes (recipe 2: still two per byte, now along K) with gate/up columns interleaved in blocks,
+ * and the scales re-laid to match.  The code outputs must be 32-byte aligned, the scale outputs
+ * 16-byte aligned.  Inputs and outputs must not overlap. */
 int moe_transform_weights(const moe_config_t *cfg, const void *w13, const void *w13_scale,
                           const void *w2, const void *w2_scale, void *w13_t, void *w13s_t,
                           void *w2_t, void *w2s_t, void *stream);
@@ -183,7 +191,8 @@ int moe_gate(const moe_config_t *cfg, const void *hidden_states, const float *no
  *   topk_weights      device fp32  [T, k]  custom routing function path); exactly one of
  *                                           router_logits and topk_idx must be non-NULL.
  *                                           The k ids of a token must be distinct, in [0, E).
- *   w13_t .. w2s_t    device, from moe_transform_weights with the same cfg fields
+ *   w13_t .. w2s_t    device, from moe_transform_weights with the same cfg fields (codes
+ *                     32-byte aligned, scales 16-byte aligned)
  *   w13_bias          device bf16 [E', 2I] or NULL (16-byte aligned; E' = num_experts + shared_experts)
  *   w2_bias           device bf16 [E', H] or NULL (16-byte aligned)
  *   y                 device bf16 [T, H], contiguous; out

@@ -2,7 +2,10 @@
 // (tcgen05.mma.kind::mxf8f6f4.block_scale): E4M3 operands with one UE8M0 power-of-two scale per
 // 32 K-elements, for rows and for weight columns ("DeepGEMM PR #371", Changes: UE8M0 scale
 // factors, 4 packed per 32-bit word, scale-factor tensors moved by TMA; "MindIE-SD Fused MoE",
-// W8A8_MXFP8).  The tensor core applies 2^(ea + ew) to every 32-deep product block itself and
+// W8A8_MXFP8).  The W4A8 recipe runs the same kernel with E2M1 weights: the weight tensor map
+// reads them packed two per byte from HBM and spreads each 16 codes over a 16-byte slot of
+// shared memory (the layout the instruction takes for 4-bit operands), the instruction
+// descriptor names E2M1 for B, and the stage expects half the weight bytes.  The tensor core applies 2^(ea + ew) to every 32-deep product block itself and
 // accumulates the whole K in TMEM, so there is no per-group promotion:
 //   mode 0: h = sum_k dec(a) 2^ea dec(w) 2^ew (+ b13); act = silu(h_gate) * h_up, requantized
 //           to E4M3 with a UE8M0 scale per 32 act columns
@@ -55,11 +58,12 @@ static_assert(kXStage % 1024 == 0, "stage alignment");
 constexpr uint32_t kXSmemBytes = XL::end + 1024;
 static_assert(kXSmemBytes <= 232448, "shared memory");
 
-// Instruction descriptor, kind::mxf8f6f4 block-scaled: E4M3 x E4M3, UE8M0 scales, K-major,
-// M = 128, N = 128; the scale-factor ids pick byte k of the 32-bit scale words.
-__device__ __forceinline__ uint32_t mx_idesc(uint32_t k) {
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: A E4M3, B E4M3 (bfmt 0) or E2M1
+// (bfmt 5), UE8M0 scales, K-major, M = 128, N = 128; the scale-factor ids pick byte k of the
+// 32-bit scale words.
+__device__ __forceinline__ uint32_t mx_idesc(uint32_t k, uint32_t bfmt) {
     return (k << 4)                       // B scale-factor id
-           | (0u << 7) | (0u << 10)       // A, B: E4M3
+           | (0u << 7) | (bfmt << 10)     // A: E4M3, B: bfmt
            | ((kXN >> 3) << 17)           // N / 8
            | (1u << 23)                   // scale format: UE8M0
            | ((kTileM >> 4) << 24)        // M / 16
@@ -167,6 +171,8 @@ __global__ void __launch_bounds__(kXThreads, 1)
                 const int brow0 = e * p.N + nb * kXN;
                 const uint8_t* sfb_src = static_cast<const uint8_t*>(p.w_scale) +
                                          (static_cast<size_t>(e) * nt + nb) * KB * kXSf;
+                // E2M1 weights arrive packed: the copy moves (and signals) half the bytes
+                const uint32_t b_bytes = p.recipe == 2 ? kXB / 2 : kXB;
                 for (int kb = 0; kb < KB; ++kb, ++it) {
                     const int s = it % kXStages;
                     if (!mbar_wait<kProducerSleepNs>(&empty[s], ((it / kXStages) & 1) ^ 1, abort_flag, p.status)) {
@@ -175,7 +181,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
                     }
                     if (fault_skip_stage(p.fault, it)) continue;   // debug builds: an injected fault
                     uint8_t* st = smem + s * kXStage;
-                    mbar_arrive_expect_tx(&full[s], kXA + kXB + kXSf);
+                    mbar_arrive_expect_tx(&full[s], kXA + b_bytes + kXSf);
                     tma_load_2d(st, &tmA, kb * kTileK, row0, &full[s]);
                     tma_load_2d(st + XL::b, &tmB, kb * kTileK, brow0, &full[s]);
                     bulk_load(st + XL::sfb, sfb_src + static_cast<size_t>(kb) * kXSf, kXSf, &full[s]);
@@ -215,6 +221,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
             // ------------------------------------------------------------------ MMA issuer
             uint32_t it = 0, tile = 0;
             bool ok = true;
+            const uint32_t bfmt = p.recipe == 2 ? 5u : 0u;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++tile) {
                 const int b = tile & 1;
                 if (!mbar_wait<kIssuerSleepNs>(&tempty[b], ((tile >> 1) & 1) ^ 1, abort_flag, p.status)) break;
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
                     sf_copy(sfb_t, sf_atom_desc(st + XL::sfb));
 #pragma unroll
                     for (uint32_t k = 0; k < 4; ++k)
-                        mma_mx(d, sw128_kmajor_desc(st + k * 32), sw128_kmajor_desc(st + XL::b + k * 32), mx_idesc(k),
+                        mma_mx(d, sw128_kmajor_desc(st + k * 32), sw128_kmajor_desc(st + XL::b + k * 32), mx_idesc(k, bfmt),
                                sfa_t, sfb_t, (kb > 0 || k > 0) ? 1u : 0u);
                     mma_commit(&empty[s]);
                 }

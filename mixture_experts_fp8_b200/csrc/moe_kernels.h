@@ -150,6 +150,6 @@ __host__ __device__ inline int w13_original_col(int r, int I, int blk) {
 }
 
 // The gate/up block of each recipe.
-__host__ __device__ inline int w13_block(int recipe) { return recipe == 1 ? 32 : 128; }
+__host__ __device__ inline int w13_block(int recipe) { return recipe != 0 ? 32 : 128; }
 
 }  // namespace moe

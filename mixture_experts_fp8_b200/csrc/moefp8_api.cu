@@ -56,8 +56,9 @@ int check_config(const moe_config_t* c) {
         return fail(MOE_ERR_INVALID_ARG, "top_k (%d) must be in [1, num_experts=%d]", c->top_k, c->num_experts);
     if (c->routing != 0 && c->routing != 1)
         return fail(MOE_ERR_INVALID_ARG, "routing must be 0 (softmax) or 1 (sigmoid), got %d", c->routing);
-    if (c->recipe != 0 && c->recipe != 1)
-        return fail(MOE_ERR_INVALID_ARG, "recipe must be 0 (fp32 per 128) or 1 (MXFP8), got %d", c->recipe);
+    if (c->recipe < 0 || c->recipe > 2)
+        return fail(MOE_ERR_INVALID_ARG, "recipe must be 0 (fp32 per 128), 1 (MXFP8) or 2 (W4A8), got %d",
+                    c->recipe);
     if (c->hidden % 128) return fail(MOE_ERR_UNSUPPORTED, "hidden (%d) must be a multiple of 128", c->hidden);
     if (c->inter % 128) return fail(MOE_ERR_UNSUPPORTED, "inter (%d) must be a multiple of 128", c->inter);
     if (c->num_experts > MOE_MAX_EXPERTS)
@@ -169,16 +170,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2D map over a row-major byte matrix [rows, cols] (cols = K, contiguous), box box_rows x 128,
-// 128-byte swizzle; rows past the end read as zero.
-int make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2D map over a row-major matrix [rows, cols] of 8-bit codes (cols = K, contiguous), box
+// box_rows x 128, 128-byte swizzle; rows past the end read as zero.  fp4: the codes are E2M1
+// packed two per byte (a row is cols / 2 bytes); each 16 codes land in a 16-byte slot of shared
+// memory (8 bytes of codes, 8 bytes of gap), the layout the tensor core takes for 4-bit operands.
+int make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                    bool fp4 = false) {
     auto fn = encode_fn();
     if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols};
+    cuuint64_t strides[1] = {fp4 ? cols / 2 : cols};
     cuuint32_t box[2] = {128, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = fn(m, fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                    const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -235,9 +240,10 @@ int moe_transformed_weights_size(const moe_config_t* cfg, size_t* w13_bytes, siz
     if (rc) return rc;
     if (!w13_bytes || !w13s_bytes || !w2_bytes || !w2s_bytes) return fail(MOE_ERR_INVALID_ARG, "NULL size pointer");
     const size_t E = cfg->num_experts + cfg->shared_experts, H = cfg->hidden, I = cfg->inter;
-    *w13_bytes = E * 2 * I * H;
+    const size_t pk = cfg->recipe == 2 ? 2 : 1;   // W4A8: two E2M1 codes per byte
+    *w13_bytes = E * 2 * I * H / pk;
     *w13s_bytes = E * (H / 128) * 2 * I * 4;
-    *w2_bytes = E * H * I;
+    *w2_bytes = E * H * I / pk;
     *w2s_bytes = E * (I / 128) * H * 4;
     return ok();
 }
@@ -249,8 +255,9 @@ int moe_transform_weights(const moe_config_t* cfg, const void* w13, const void* 
     if (!w13 || !w13_scale || !w2 || !w2_scale || !w13_t || !w13s_t || !w2_t || !w2s_t)
         return fail(MOE_ERR_INVALID_ARG, "moe_transform_weights: NULL pointer");
     if (!aligned(w13_scale, 4) || !aligned(w2_scale, 4) || !aligned(w13s_t, 16) || !aligned(w2s_t, 16) ||
-        !aligned(w13_t, 16) || !aligned(w2_t, 16))
-        return fail(MOE_ERR_INVALID_ARG, "moe_transform_weights: misaligned buffer (outputs need 16 bytes)");
+        !aligned(w13_t, 32) || !aligned(w2_t, 32))
+        return fail(MOE_ERR_INVALID_ARG,
+                    "moe_transform_weights: misaligned buffer (transformed codes need 32 bytes, scales 16)");
     DeviceInfo di;
     if ((rc = device_info(&di))) return rc;
     moe::TransformArgs a{static_cast<const uint8_t*>(w13), w13_scale, static_cast<const uint8_t*>(w2), w2_scale,
@@ -306,13 +313,14 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     if ((router_logits == nullptr) == (topk_idx == nullptr))
         return fail(MOE_ERR_INVALID_ARG, "moe_forward: pass exactly one of router_logits and topk_idx");
     if (topk_idx && !topk_weights) return fail(MOE_ERR_INVALID_ARG, "moe_forward: topk_idx needs topk_weights");
-    if (!aligned(hidden_states, 16) || !aligned(y, 16) || !aligned(w13_t, 16) || !aligned(w2_t, 16) ||
+    if (!aligned(hidden_states, 16) || !aligned(y, 16) || !aligned(w13_t, 32) || !aligned(w2_t, 32) ||
         !aligned(w13s_t, 16) || !aligned(w2s_t, 16) || !aligned(workspace, 256) ||
         (router_logits && !aligned(router_logits, 4)) || (topk_idx && !aligned(topk_idx, 4)) ||
         (topk_weights && !aligned(topk_weights, 4)) || (w13_bias && !aligned(w13_bias, 16)) ||
         (w2_bias && !aligned(w2_bias, 16)) || (expert_counts && !aligned(expert_counts, 4)))
         return fail(MOE_ERR_INVALID_ARG,
-                    "moe_forward: misaligned buffer (hidden_states, y, weights and biases need 16 bytes, workspace 256)");
+                    "moe_forward: misaligned buffer (hidden_states, y, biases and scales need 16 bytes, "
+                    "weight codes 32, workspace 256)");
     moe_workspace_layout_t L;
     layout_of(cfg, &L);
     if (workspace_bytes < L.total)
@@ -335,16 +343,17 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     // MXFP8 runs the block-scaled tensor-core kernels.  fp32 scales: few rows per expert (decode)
     // take the swap-AB kernels, weights as the M operand, else the wide kernels; both compute every
     // row with the same operations, so the choice does not change bits.
-    const bool mx = cfg->recipe == 1;
+    const bool mx = cfg->recipe != 0;     // MXFP8 and W4A8: the block-scaled kernels
+    const bool fp4 = cfg->recipe == 2;
     const bool narrow = !mx && A <= moe::kNarrowRowsPerExpert * ET;
     CUtensorMap tm_x, tm_w13, tm_act, tm_w2;
     const uint32_t tok_box = narrow ? 16 : moe::kTileM;
     const uint32_t w13_box = mx ? 128 : narrow ? moe::kTileN : moe::gemm_weight_box(0);
     const uint32_t w2_box = mx ? 128 : narrow ? moe::kTileN : moe::gemm_weight_box(1);
     if ((rc = make_kmajor_map(&tm_x, at(L.xq), A, H, tok_box))) return rc;
-    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(ET) * 2 * I, H, w13_box))) return rc;
+    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(ET) * 2 * I, H, w13_box, fp4))) return rc;
     if ((rc = make_kmajor_map(&tm_act, at(L.act_q), A, I, tok_box))) return rc;
-    if ((rc = make_kmajor_map(&tm_w2, w2_t, static_cast<uint64_t>(ET) * H, I, w2_box))) return rc;
+    if ((rc = make_kmajor_map(&tm_w2, w2_t, static_cast<uint64_t>(ET) * H, I, w2_box, fp4))) return rc;
 
     cudaEvent_t* ev = nullptr;
     if (prof && (rc = prof_next(prof, &ev))) return rc;

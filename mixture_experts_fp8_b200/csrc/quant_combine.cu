@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
             continue;
         }
         *reinterpret_cast<uint32_t*>(a.xq + static_cast<size_t>(r) * a.H + cb * 128 + 4 * lane) = q;
-        if (a.recipe == 1 && (lane & 7) == 0)
+        if (a.recipe != 0 && (lane & 7) == 0)
             static_cast<uint8_t*>(a.xs)[(static_cast<size_t>(cb) * a.a_pad + r) * 4 + (lane >> 3)] = e8;
     }
     // fp32 scales: lane j stores the scale of the token's j-th row (one instruction for up to 32)
@@ -121,6 +121,9 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
 //   recipe 0: fp32 [E, K/128, N] -> [E, K/128, N'] (columns permuted like the codes)
 //   recipe 1: UE8M0 [E, K/32, N] -> 512-byte scale-factor atoms [E, N/128, K/128] for the
 //             block-scaled tensor core (see gemm_mx.cu)
+//   recipe 2 (W4A8): E2M1 codes packed two per byte along N, [E, K, N/2] -> packed two per
+//             byte along K, [E, N', K/2] (the lower K in the low nibble; k_transpose_nibbles),
+//             scales as recipe 1
 // ("MATE Mega MoE", transform_weights_for_mega_moe; "DeepGEMM PR #371", 4-packed UE8M0.)
 __global__ void __launch_bounds__(256) k_transpose_codes(const uint8_t* src, uint8_t* dst, int K,
                                                         int N, int interleave_I, int blk) {
@@ -140,6 +143,35 @@ __global__ void __launch_bounds__(256) k_transpose_codes(const uint8_t* src, uin
         if (n < N && k < K) {
             const int row = interleave_I ? w13_interleaved_row(n, interleave_I, blk) : n;
             d[static_cast<size_t>(row) * K + k] = tile[kk][nn];
+        }
+    }
+}
+
+// E2M1 codes: a 64 x 64 tile of [K, N] codes (N packed in pairs) is unpacked into shared
+// memory, then written back K-major with K packed in pairs.
+__global__ void __launch_bounds__(256) k_transpose_nibbles(const uint8_t* src, uint8_t* dst, int K,
+                                                          int N, int interleave_I, int blk) {
+    __shared__ uint8_t tile[64][65];
+    const int e = blockIdx.z;
+    const int k0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+    const uint8_t* s = src + static_cast<size_t>(e) * K * (N / 2);
+    uint8_t* d = dst + static_cast<size_t>(e) * N * (K / 2);
+    for (int i = threadIdx.x; i < 64 * 32; i += 256) {          // 64 rows x 32 bytes
+        const int kk = i / 32, jj = i % 32;
+        if (k0 + kk < K && n0 + 2 * jj < N) {
+            const uint8_t b = s[static_cast<size_t>(k0 + kk) * (N / 2) + n0 / 2 + jj];
+            tile[kk][2 * jj] = b & 15;
+            tile[kk][2 * jj + 1] = b >> 4;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 64 * 32; i += 256) {          // 64 columns x 32 bytes
+        const int nn = i / 32, jj = i % 32;
+        const int n = n0 + nn, k = k0 + 2 * jj;
+        if (n < N && k < K) {
+            const int row = interleave_I ? w13_interleaved_row(n, interleave_I, blk) : n;
+            d[static_cast<size_t>(row) * (K / 2) + k / 2] =
+                static_cast<uint8_t>(tile[2 * jj][nn] | (tile[2 * jj + 1][nn] << 4));
         }
     }
 }
@@ -183,9 +215,9 @@ __global__ void k_transform_scales(const void* src, void* dst, int E, int K, int
 
 cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s) {
     const int H = a.H, I = a.I, E = a.E;
-    k_transpose_codes<<<dim3((2 * I + 63) / 64, (H + 63) / 64, E), 256, 0, s>>>(a.w13, a.w13_t, H, 2 * I, I,
-                                                                                 w13_block(a.recipe));
-    k_transpose_codes<<<dim3((H + 63) / 64, (I + 63) / 64, E), 256, 0, s>>>(a.w2, a.w2_t, I, H, 0, 1);
+    auto codes = a.recipe == 2 ? k_transpose_nibbles : k_transpose_codes;
+    codes<<<dim3((2 * I + 63) / 64, (H + 63) / 64, E), 256, 0, s>>>(a.w13, a.w13_t, H, 2 * I, I, w13_block(a.recipe));
+    codes<<<dim3((H + 63) / 64, (I + 63) / 64, E), 256, 0, s>>>(a.w2, a.w2_t, I, H, 0, 1);
     k_transform_scales<<<1024, 256, 0, s>>>(a.w13s, a.w13s_t, E, H, 2 * I, a.recipe, I);
     k_transform_scales<<<1024, 256, 0, s>>>(a.w2s, a.w2s_t, E, I, H, a.recipe, 0);
     return cudaGetLastError();

@@ -76,7 +76,8 @@ def test_valid_configs_and_sizes():
         assert all(v % 1024 == 0 for k, v in lay.items() if k not in ("total", "scale_rows"))
         assert lay["scale_rows"] >= A and lay["scale_rows"] % 4 == 0
         w13, w13s, w2, w2s = moe.transformed_weights_size(c)
-        assert w13 == s.num_experts * s.hidden * 2 * s.inter and w2 == s.num_experts * s.inter * s.hidden
+        pk = 2 if s.recipe == 2 else 1          # W4A8: two E2M1 codes per byte
+        assert w13 * pk == s.num_experts * s.hidden * 2 * s.inter and w2 * pk == s.num_experts * s.inter * s.hidden
         assert w13s == s.num_experts * (s.hidden // 128) * 2 * s.inter * 4
 
 

@@ -9,7 +9,8 @@ inputs, for every step of the layer.
 
 Sizes: the tiny problem and small ragged problems in full (several tiles, ragged tails, empty
 experts); the four full-size problems with routing, permutation and quantization in full and y
-on seeded token samples (a row's bits do not depend on the other rows).
+on seeded token samples (a row's bits do not depend on the other rows).  The W4A8 recipe (E2M1
+weights) runs on the decode and prefill shapes, the small random problems and the edge shapes.
 """
 import numpy as np
 import pytest
@@ -22,8 +23,10 @@ from _helpers import (GpuProblem, assert_y_close, bits, check_routing, oracle_cf
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["tiny", "decode", "prefill", "skewed", "large"]
-SAMPLE_TOKENS = {"tiny": None, "decode": None, "skewed": 384, "prefill": 48, "large": 96}
+FULL = ["tiny", "decode", "prefill", "skewed", "large", "decode_w4a8", "prefill_w4a8"]
+SAMPLE_TOKENS = {"tiny": None, "decode": None, "skewed": 384, "prefill": 48, "large": 96,
+                 "decode_w4a8": None, "prefill_w4a8": 48}
+ON_GPU = ("prefill", "large", "prefill_w4a8")     # inputs drawn on the device (their size)
 
 
 @pytest.fixture(scope="module")
@@ -32,7 +35,7 @@ def problems():
 
     def get(name):
         if name not in cache:
-            dev = "cuda" if name in ("prefill", "large") else "cpu"
+            dev = "cuda" if name in ON_GPU else "cpu"
             prob = synth.make_problem(name, device=dev)
             gp = GpuProblem(prob)
             cache[name] = (gp, oracle_inputs(prob))
@@ -151,9 +154,9 @@ def test_forward_output(problems, name):
     print(f"{name}: {m}")
 
 
-@pytest.mark.parametrize("seed", range(8))
-def test_forward_random_small(seed):
-    shape = synth.random_shape(seed)
+@pytest.mark.parametrize("seed,recipe", [(s, None) for s in range(8)] + [(s, 2) for s in range(8, 12)])
+def test_forward_random_small(seed, recipe):
+    shape = synth.random_shape(seed) if recipe is None else synth.random_shape(seed, recipe=recipe)
     prob = synth.make_problem(shape)
     gp = GpuProblem(prob)
     ni = oracle_inputs(prob)
@@ -171,7 +174,7 @@ def test_forward_random_small(seed):
     dict(num_tokens=50, hidden=384, inter=640, num_experts=5, top_k=2),   # 3 K stages, odd N tiles
     dict(num_tokens=33, hidden=128, inter=128, num_experts=64, top_k=3),  # many empty experts
 ])
-@pytest.mark.parametrize("recipe", [0, 1])
+@pytest.mark.parametrize("recipe", [0, 1, 2])
 def test_forward_edge_shapes(over, recipe):
     base = synth.Shape("edge", 8, 256, 256, 4, 2, renormalize=1, recipe=recipe, seed=77, biases=True)
     from dataclasses import replace
