@@ -230,6 +230,9 @@ def main():
                     help="override the problem's token count (reduced cases for profiler captures)")
     ap.add_argument("--shared-expert", action="store_true",
                     help="add a shared expert (every token, weight 1) to the problem")
+    ap.add_argument("--gate", action="store_true",
+                    help="start each step from the gate (RMSNorm + router matmul + top-k, moe_gate) on "
+                         "the bf16 hidden states instead of from precomputed router logits")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -270,10 +273,23 @@ def main():
     y = torch.empty((shape.num_tokens, shape.hidden), dtype=torch.bfloat16, device=dev)
     counts = torch.zeros(shape.num_experts + shape.shared_experts, dtype=torch.int32, device=dev)
 
-    def step(profile=None):
-        moe.forward(cfg, d.x, weights, router_logits=d.logits, per_expert_scale=d.per_expert_scale,
-                    w13_bias=d.w13_bias, w2_bias=d.w2_bias, y=y, expert_counts=counts, workspace=ws,
-                    profile=profile)
+    if args.gate:
+        norm_w, router_w, eps = (t.to(dev) if torch.is_tensor(t) else t for t in synth.make_gate(shape))
+        g_logits = torch.empty((shape.num_tokens, shape.num_experts), dtype=torch.float32, device=dev)
+        g_idx = torch.empty((shape.num_tokens, shape.top_k), dtype=torch.int32, device=dev)
+        g_w = torch.empty((shape.num_tokens, shape.top_k), dtype=torch.float32, device=dev)
+
+    def step(profile=None, x=None):
+        x = d.x if x is None else x
+        if args.gate:      # the gate replaces the router; the forward takes its routing
+            moe.gate(cfg, x, norm_w, router_w, eps, per_expert_scale=d.per_expert_scale, logits=g_logits,
+                     topk_idx=g_idx, topk_weights=g_w)
+            moe.forward(cfg, x, weights, topk_idx=g_idx, topk_weights=g_w, w13_bias=d.w13_bias,
+                        w2_bias=d.w2_bias, y=y, expert_counts=counts, workspace=ws, profile=profile)
+        else:
+            moe.forward(cfg, x, weights, router_logits=d.logits, per_expert_scale=d.per_expert_scale,
+                        w13_bias=d.w13_bias, w2_bias=d.w2_bias, y=y, expert_counts=counts, workspace=ws,
+                        profile=profile)
 
     for _ in range(args.warmup):
         step()
@@ -325,10 +341,27 @@ def main():
 
     def e2e_step():
         x_d.copy_(x_h, non_blocking=True)
-        l_d.copy_(l_h, non_blocking=True)
-        moe.forward(cfg, x_d, weights, router_logits=l_d, per_expert_scale=d.per_expert_scale,
-                    w13_bias=d.w13_bias, w2_bias=d.w2_bias, y=y, workspace=ws)
+        if args.gate:          # the gate's input is x alone
+            step(x=x_d)
+        else:
+            l_d.copy_(l_h, non_blocking=True)
+            moe.forward(cfg, x_d, weights, router_logits=l_d, per_expert_scale=d.per_expert_scale,
+                        w13_bias=d.w13_bias, w2_bias=d.w2_bias, y=y, workspace=ws)
         y_h.copy_(y, non_blocking=True)
+
+    gate_ms = None
+    if args.gate:              # the gate kernel alone, CUDA events on the launch stream
+        for _ in range(args.warmup):
+            moe.gate(cfg, d.x, norm_w, router_w, eps, per_expert_scale=d.per_expert_scale, logits=g_logits,
+                     topk_idx=g_idx, topk_weights=g_w)
+        q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        q0.record()
+        for _ in range(args.steps):
+            moe.gate(cfg, d.x, norm_w, router_w, eps, per_expert_scale=d.per_expert_scale, logits=g_logits,
+                     topk_idx=g_idx, topk_weights=g_w)
+        q1.record()
+        torch.cuda.synchronize()
+        gate_ms = q0.elapsed_time(q1) / args.steps
 
     for _ in range(args.warmup):
         e2e_step()
@@ -356,6 +389,8 @@ def main():
         per_step_s = ms / 1e3 / args.steps
         fl = flops(shape, A)
         alg = algorithmic_bytes(shape, active)
+        if args.gate:          # + the router and norm weights (the logits are written instead of read)
+            alg += 4 * shape.num_experts * shape.hidden + 4 * shape.hidden
         g1_ms = stage_ms["gemm1_swiglu_requant"] / max(calls, 1)
         g2_ms = stage_ms["gemm2"] / max(calls, 1)
         g1_bytes = gemm1_bytes(shape, active)
@@ -381,7 +416,9 @@ def main():
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
-            "config": {"workload": describe(shape), "tokens_per_step": shape.num_tokens,
+            "config": {"workload": describe(shape) + ("; from bf16 hidden states through the fused gate "
+                                                      "(RMSNorm + router matmul + top-k)" if args.gate else ""),
+                       "tokens_per_step": shape.num_tokens,
                        "active_experts": active, "parallelism": f"replicas x{world}",
                        "l2": "no flush; the step streams the FP8 weights, larger than L2" if alg > 126e6
                              else "working set fits L2 (latency-bound)"},
@@ -394,9 +431,16 @@ def main():
             "gemm2": {"ms": g2_ms, "GB/s": gemm2_bytes(shape, active) / (g2_ms / 1e3) / 1e9},
             "clocks": clocks, "gpu_launches": kernels_per_step(A) * args.steps, "status": status,
             "e2e": {"value": world * shape.num_tokens * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": x_h.numel() * 2 + l_h.numel() * 4,
+                    "h2d_bytes_per_step": x_h.numel() * 2 + (0 if args.gate else l_h.numel() * 4),
                     "d2h_bytes_per_step": y_h.numel() * 2},
         }
+        if args.gate:
+            T, H, E, k = shape.num_tokens, shape.hidden, shape.num_experts, shape.top_k
+            gbytes = 2 * T * H + 4 * H + 4 * E * H + 4 * T * E + 8 * T * k
+            line["gate"] = {"kernel": "k_gate", "ms_per_launch": gate_ms, "algorithmic_bytes": gbytes,
+                            "GB/s": gbytes / (gate_ms / 1e3) / 1e9,
+                            "note": "stages_ms covers the forward after the gate (its route stage is "
+                                    "empty: the routing comes from the gate)"}
         if world == 1 and not args.no_cpu_baseline:
             n = {"tiny": 16, "decode": 64, "skewed": 64, "prefill": 4, "large": 16}.get(shape.name, 8)
             cpu_prob = prob if prob.x.device.type == "cpu" else None

@@ -164,18 +164,19 @@ int moe_workspace_layout(const moe_config_t *cfg, moe_workspace_layout_t *layout
 int moe_route(const moe_config_t *cfg, const float *router_logits, const float *per_expert_scale,
               int32_t *topk_idx, float *topk_weights, void *stream);
 
-/* The gate in front of the router, fused with it ("mlx_native ops/moe_gate.rs": RMS-Norm of
- * the hidden state, the router matmul, then top-K + softmax + per-expert scale):
+/* The gate in front of the router ("mlx_native ops/moe_gate.rs": RMS-Norm of the hidden state,
+ * the router matmul, then top-K + softmax + per-expert scale):
  *   logits[t, e] = sum_h ( x[t,h] / sqrt(mean_h x[t,h]^2 + rms_eps) * norm_weight[h] ) * router_weight[e, h]
- * in fp32 (fixed summation order: a token's logits do not depend on the other tokens), then the
- * router of moe_route on those logits with cfg's routing fields.
+ * in fp32, computed as r_t * sum_h (x[t,h] * norm_weight[h]) * router_weight[e,h] with the sum in
+ * ascending h (a token's logits do not depend on the other tokens or on T), then the router of
+ * moe_route on those logits with cfg's routing fields.
  *   hidden_states     device bf16 [T, H], 16-byte aligned
- *   norm_weight       device fp32 [H]
+ *   norm_weight       device fp32 [H], 16-byte aligned
  *   router_weight     device fp32 [E, H] row-major, 16-byte aligned (E = cfg->num_experts)
  *   per_expert_scale  device fp32 [E] or NULL
  *   logits            device fp32 [T, E]  out
  *   topk_idx          device int32 [T, k] out;  topk_weights device fp32 [T, k] out
- * One launch.  Limit (MOE_ERR_UNSUPPORTED): hidden <= 12288.  Feed topk_idx/topk_weights to
+ * Two launches (the tiled router matmul, then the router).  Feed topk_idx/topk_weights to
  * moe_forward to run the layer on them. */
 int moe_gate(const moe_config_t *cfg, const void *hidden_states, const float *norm_weight,
              const float *router_weight, float rms_eps, const float *per_expert_scale, float *logits,

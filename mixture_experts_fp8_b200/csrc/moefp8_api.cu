@@ -436,12 +436,12 @@ int moe_gate(const moe_config_t* cfg, const void* hidden_states, const float* no
     if (rc) return rc;
     if (!hidden_states || !norm_weight || !router_weight || !logits || !topk_idx || !topk_weights)
         return fail(MOE_ERR_INVALID_ARG, "moe_gate: NULL pointer");
-    if (!aligned(hidden_states, 16) || !aligned(router_weight, 16) || !aligned(norm_weight, 4) ||
+    if (!aligned(hidden_states, 16) || !aligned(router_weight, 16) || !aligned(norm_weight, 16) ||
         !aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_weights, 4) ||
         (per_expert_scale && !aligned(per_expert_scale, 4)))
-        return fail(MOE_ERR_INVALID_ARG, "moe_gate: misaligned buffer (hidden_states and router_weight need 16 bytes)");
+        return fail(MOE_ERR_INVALID_ARG,
+                    "moe_gate: misaligned buffer (hidden_states, norm_weight and router_weight need 16 bytes)");
     if (!(rms_eps >= 0.0f)) return fail(MOE_ERR_INVALID_ARG, "moe_gate: rms_eps must be >= 0");
-    if (cfg->hidden > 12288) return fail(MOE_ERR_UNSUPPORTED, "moe_gate: hidden (%d) exceeds 12288", cfg->hidden);
     DeviceInfo di;
     if ((rc = device_info(&di))) return rc;
     moe::GateArgs g{static_cast<const __nv_bfloat16*>(hidden_states), norm_weight, router_weight, logits, rms_eps,

@@ -94,3 +94,21 @@ def test_gate_routing_drives_the_layer_like_router_logits():
     y2 = bits(gp.forward(logits=lg))
     assert gp.status() == 0
     assert np.array_equal(y1, y2)
+
+
+def test_gate_logits_same_for_both_tile_shapes():
+    """A large batch takes the 64 x 64 tiles, a few tokens the 16 x 16 tiles: every logit is still
+    the same sum in the same order, so a token's logits are bit-identical either way."""
+    import mixture_experts_fp8_b200 as moe
+    shape = synth.Shape("gtiles", 2400, 256, 128, 256, 8, renormalize=1, seed=43)   # 38 x 4 blocks of 64 x 64
+    prob, nw, rw, eps = _gate_inputs(shape)
+    cfg = moe.Config(**shape.cfg())
+    x = prob.x.cuda()
+    lg, _, _ = moe.gate(cfg, x, nw.cuda(), rw.cuda(), eps)
+    sel = torch.tensor([2399, 0, 1234, 7], device="cuda")
+    cs = moe.Config(**replace(shape, num_tokens=4).cfg())
+    ls, _, _ = moe.gate(cs, x[sel].contiguous(), nw.cuda(), rw.cuda(), eps)
+    torch.cuda.synchronize()
+    assert torch.equal(ls, lg[sel])
+    ref = oracle.gate_logits(prob.numpy_inputs()["x"][[2399, 0, 1234, 7]], nw.numpy(), rw.numpy(), eps)
+    assert np.max(np.abs(ls.cpu().numpy() - ref)) / np.max(np.abs(ref)) <= LOGIT_TOL
