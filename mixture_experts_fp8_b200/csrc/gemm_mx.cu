@@ -194,18 +194,51 @@ __global__ void __launch_bounds__(kXThreads, 1)
         }
     } else if (warp == 2) {
         // ---------------------------------------------------------------------- row-scale atoms
-        // lane i writes the atom's row i: the scale words of tile rows i, 32+i, 64+i, 96+i.
-        uint32_t it = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        // lane i writes the atom's row i: the scale words of tile rows i, 32+i, 64+i, 96+i.  The
+        // words are gathered kSfAhead stages ahead of the stage being written (a register ring)
+        // by an iterator that decodes each unit once, so the gather's global-load latency is not
+        // paid once per stage.
+        constexpr int kSfAhead = 2;
+        const int my_units = total_units > static_cast<int>(blockIdx.x)
+                                 ? (total_units - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1
+                                 : 0;
+        const int n_stages = my_units * KB;           // stages this CTA runs, in order
+        // the gather's own position (unit, stage, first row), advanced one stage per call
+        int gu = static_cast<int>(blockIdx.x), gkb = 0, grow0 = 0;
+        if (gu < total_units) {
             int e, nb, mb;
-            decode_unit_x(u, nt, s_tstart, p.E, e, nb, mb);
-            const int row0 = s_off[e] + mb * kTileM;
-            for (int kb = 0; kb < KB; ++kb, ++it) {
+            decode_unit_x(gu, nt, s_tstart, p.E, e, nb, mb);
+            grow0 = s_off[e] + mb * kTileM;
+        }
+        auto gather = [&]() {                         // the next stage's scale words (zeros past the end)
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (gu < total_units) {
+                const uint32_t* src = static_cast<const uint32_t*>(p.a_scale) + static_cast<size_t>(gkb) * p.a_pad + grow0;
+                w = make_uint4(__ldg(src + lane), __ldg(src + 32 + lane), __ldg(src + 64 + lane), __ldg(src + 96 + lane));
+                if (++gkb == KB) {
+                    gkb = 0;
+                    gu += static_cast<int>(gridDim.x);
+                    if (gu < total_units) {
+                        int e, nb, mb;
+                        decode_unit_x(gu, nt, s_tstart, p.E, e, nb, mb);
+                        grow0 = s_off[e] + mb * kTileM;
+                    }
+                }
+            }
+            return w;
+        };
+        uint4 ring[kSfAhead];
+#pragma unroll
+        for (int d = 0; d < kSfAhead; ++d) ring[d] = gather();
+        bool ok = true;
+        for (int base = 0; base < n_stages && ok; base += kSfAhead) {
+#pragma unroll
+            for (int d = 0; d < kSfAhead; ++d) {
+                const int it = base + d;
+                if (it >= n_stages) break;
+                const uint4 w = ring[d];
+                ring[d] = gather();
                 const int s = it % kXStages;
-                const uint32_t* src = static_cast<const uint32_t*>(p.a_scale) + static_cast<size_t>(kb) * p.a_pad + row0;
-                const uint4 w = make_uint4(__ldg(src + lane), __ldg(src + 32 + lane), __ldg(src + 64 + lane),
-                                           __ldg(src + 96 + lane));
                 if (!mbar_wait<kProducerSleepNs>(&empty[s], ((it / kXStages) & 1) ^ 1, abort_flag, p.status)) {
                     ok = false;
                     break;
