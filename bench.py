@@ -230,6 +230,8 @@ def main():
                     help="override the problem's token count (reduced cases for profiler captures)")
     ap.add_argument("--shared-expert", action="store_true",
                     help="add a shared expert (every token, weight 1) to the problem")
+    ap.add_argument("--recipe", type=int, default=None, choices=[0, 1, 2],
+                    help="run the problem with another quantization recipe (0 fp32 per 128, 1 MXFP8, 2 W4A8)")
     ap.add_argument("--gate", action="store_true",
                     help="start each step from the gate (RMSNorm + router matmul + top-k, moe_gate) on "
                          "the bf16 hidden states instead of from precomputed router logits")
@@ -245,6 +247,9 @@ def main():
     if args.shared_expert:
         from dataclasses import replace
         shape = replace(shape, shared_experts=1)
+    if args.recipe is not None and args.recipe != shape.recipe:
+        from dataclasses import replace
+        shape = replace(shape, recipe=args.recipe, name=f"{shape.name}_r{args.recipe}")
 
     if args.impl == "reference":
         reference_arm(args, shape, rank)
@@ -261,7 +266,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     dev = f"cuda:{local}"
-    big = shape.name in ("prefill", "large", "prefill_w4a8")     # inputs drawn on the device
+    # big problems (prefill, large): inputs drawn on the device, the fp32 weights freed after the transform
+    big = shape.num_experts * shape.hidden * shape.inter >= 500_000_000
     gen_dev = dev if big else "cpu"
     prob = synth.make_problem(shape, device=gen_dev)
     d = prob.to(dev)
@@ -402,11 +408,11 @@ def main():
                     "frac": g1_tflops / fp8_peak}
         else:
             roof = {"bound": "hbm", "achieved": g1_gbs, "peak": hbm, "unit": "GB/s", "frac": g1_gbs / hbm}
-        # the library's kernel choice: MXFP8 -> block-scaled kernel; fp32 scales -> swap-AB narrow
-        # kernel at <= 32 routed rows per expert, else the wide kernel
-        kname = ("k_grouped_gemm_mx" if shape.recipe != 0 else
-                 "k_grouped_gemm_narrow" if A <= 32 * (shape.num_experts + shape.shared_experts)
-                 else "k_grouped_gemm")
+        # the library's kernel choice: at most 32 routed rows per expert on average -> the swap-AB
+        # kernels (fp32 scales: narrow; MXFP8 / W4A8: mx_narrow), else the wide ones
+        few = A <= 32 * (shape.num_experts + shape.shared_experts)
+        kname = ("k_grouped_gemm_mx_narrow" if few else "k_grouped_gemm_mx") if shape.recipe != 0 else \
+                ("k_grouped_gemm_narrow" if few else "k_grouped_gemm")
         roof.update({"kernel": kname + "<gate+up>",
                      "traffic": traffic_for("gemm1", shape.name),
                      "peak_source": f"{pk_kind} ({'sustained bf16 x2 for fp8' if compute_bound else 'copy'})",

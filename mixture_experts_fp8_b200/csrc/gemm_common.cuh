@@ -62,4 +62,43 @@ __device__ __forceinline__ void add_bias32(float* acc, const __nv_bfloat16* bias
     for (int v = 0; v < 4; ++v) add_bias8(acc + 8 * v, ld_nc_u4(b4 + v));
 }
 
+// ------------------------------------------------------------------ block-scaled (MX) MMA pieces
+// Instruction descriptor, kind::mxf8f6f4 block-scaled, UE8M0 scale factors, both operands
+// K-major: afmt / bfmt 0 = E4M3, 5 = E2M1; the scale-factor ids pick byte k of the 32-bit scale
+// words (the k-th 32-deep block of a 128-deep stage).
+__device__ __forceinline__ uint32_t mx_block_idesc(uint32_t k, uint32_t afmt, uint32_t bfmt, int M, int N) {
+    return (k << 4)                                       // B scale-factor id
+           | (afmt << 7) | (bfmt << 10)                   // A, B element formats
+           | (static_cast<uint32_t>(N >> 3) << 17)        // N / 8
+           | (1u << 23)                                   // scale format: UE8M0
+           | (static_cast<uint32_t>(M >> 4) << 24)        // M / 16
+           | (k << 29);                                   // A scale-factor id
+}
+
+__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Shared-memory descriptor of one scale-factor atom: 32 rows of 16 bytes, contiguous, no swizzle
+// (8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(128 >> 4) << 32;   // stride between 8-row core matrices
+    d |= static_cast<uint64_t>(1) << 46;           // descriptor version
+    return d;                                       // layout type 0: no swizzle
+}
+
+// Copy one scale-factor atom (32 rows x 16 bytes) into 4 TMEM columns of every lane quadrant:
+// row i's word c lands in lane i, column c.  The MMA reads the scale of row r from lane r % 32,
+// column r / 32, byte = its scale-factor id.
+__device__ __forceinline__ void sf_copy(uint32_t tmem_col_addr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem_col_addr), "l"(sdesc) : "memory");
+}
+
 }  // namespace moe

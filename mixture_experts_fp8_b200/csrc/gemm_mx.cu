@@ -58,41 +58,6 @@ static_assert(kXStage % 1024 == 0, "stage alignment");
 constexpr uint32_t kXSmemBytes = XL::end + 1024;
 static_assert(kXSmemBytes <= 232448, "shared memory");
 
-// Instruction descriptor, kind::mxf8f6f4 block-scaled: A E4M3, B E4M3 (bfmt 0) or E2M1
-// (bfmt 5), UE8M0 scales, K-major, M = 128, N = 128; the scale-factor ids pick byte k of the
-// 32-bit scale words.
-__device__ __forceinline__ uint32_t mx_idesc(uint32_t k, uint32_t bfmt) {
-    return (k << 4)                       // B scale-factor id
-           | (0u << 7) | (bfmt << 10)     // A: E4M3, B: bfmt
-           | ((kXN >> 3) << 17)           // N / 8
-           | (1u << 23)                   // scale format: UE8M0
-           | ((kTileM >> 4) << 24)        // M / 16
-           | (k << 29);                   // A scale-factor id
-}
-
-__device__ __forceinline__ void mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
-        : "memory");
-}
-
-// Shared-memory descriptor of one scale-factor atom: 32 rows of 16 bytes, contiguous, no swizzle
-// (8-row core matrices 128 bytes apart).
-__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t smem_addr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>(128 >> 4) << 32;   // stride between 8-row core matrices
-    d |= static_cast<uint64_t>(1) << 46;           // descriptor version
-    return d;                                       // layout type 0: no swizzle
-}
-
-__device__ __forceinline__ void sf_copy(uint32_t tmem_col_addr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(tmem_col_addr), "l"(sdesc) : "memory");
-}
-
 __device__ __forceinline__ void decode_unit_x(int u, int nt, const int* tstart, int E, int& e, int& nb, int& mb) {
     int lo = 0, hi = E - 1;
     while (lo < hi) {
@@ -275,7 +240,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
                     sf_copy(sfb_t, sf_atom_desc(st + XL::sfb));
 #pragma unroll
                     for (uint32_t k = 0; k < 4; ++k)
-                        mma_mx(d, sw128_kmajor_desc(st + k * 32), sw128_kmajor_desc(st + XL::b + k * 32), mx_idesc(k, bfmt),
+                        mma_mx(d, sw128_kmajor_desc(st + k * 32), sw128_kmajor_desc(st + XL::b + k * 32), mx_block_idesc(k, 0u, bfmt, kTileM, kXN),
                                sfa_t, sfb_t, (kb > 0 || k > 0) ? 1u : 0u);
                     mma_commit(&empty[s]);
                 }

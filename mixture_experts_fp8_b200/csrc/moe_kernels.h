@@ -123,6 +123,9 @@ cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtenso
                         int num_sms, cudaStream_t s);
 cudaError_t launch_gemm_mx(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
                            cudaStream_t s);
+cudaError_t launch_gemm_mx_narrow(const GemmArgs& a, const CUtensorMap& tmW, const CUtensorMap& tmT, int num_sms,
+                                  cudaStream_t s);
+uint32_t gemm_mx_narrow_tokens();
 cudaError_t launch_gemm_narrow(const GemmArgs& a, const CUtensorMap& tmW, const CUtensorMap& tmT,
                                int num_sms, cudaStream_t s);
 // The narrow (swap-AB) GEMMs take problems averaging at most this many routed rows per expert.

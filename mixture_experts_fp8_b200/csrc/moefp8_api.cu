@@ -338,16 +338,15 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     const int32_t* idx = topk_idx ? topk_idx : static_cast<const int32_t*>(at(L.topk_idx));
     const float* wts = topk_idx ? topk_weights : static_cast<const float*>(at(L.topk_weights));
 
-    // Few rows per expert (decode): the swap-AB kernels, weights as the M operand; else the wide
-    // kernels.  Both compute every row with the same operations, so the choice does not change bits.
-    // MXFP8 runs the block-scaled tensor-core kernels.  fp32 scales: few rows per expert (decode)
-    // take the swap-AB kernels, weights as the M operand, else the wide kernels; both compute every
-    // row with the same operations, so the choice does not change bits.
+    // Few rows per expert (decode, at most kNarrowRowsPerExpert on average) take the swap-AB
+    // kernels, the weights as the M operand; else the wide kernels.  fp32 scales: both compute every
+    // row with the same operations in the same order.  MXFP8 and W4A8 run the block-scaled tensor
+    // core kernels, swap-AB (gemm_mx_narrow.cu) or wide (gemm_mx.cu).
     const bool mx = cfg->recipe != 0;     // MXFP8 and W4A8: the block-scaled kernels
     const bool fp4 = cfg->recipe == 2;
-    const bool narrow = !mx && A <= moe::kNarrowRowsPerExpert * ET;
+    const bool narrow = A <= moe::kNarrowRowsPerExpert * ET;
     CUtensorMap tm_x, tm_w13, tm_act, tm_w2;
-    const uint32_t tok_box = narrow ? 16 : moe::kTileM;
+    const uint32_t tok_box = !narrow ? moe::kTileM : mx ? moe::gemm_mx_narrow_tokens() : 16;
     const uint32_t w13_box = mx ? 128 : narrow ? moe::kTileN : moe::gemm_weight_box(0);
     const uint32_t w2_box = mx ? 128 : narrow ? moe::kTileN : moe::gemm_weight_box(1);
     if ((rc = make_kmajor_map(&tm_x, at(L.xq), A, H, tok_box))) return rc;
@@ -403,9 +402,10 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     g1.act_s = at(L.act_s);
     g1.status = status;
     g1.fault = take_armed_fault();
-    MOE_CUDA_TRY(mx       ? moe::launch_gemm_mx(g1, tm_x, tm_w13, di.sms, s)
-                 : narrow ? moe::launch_gemm_narrow(g1, tm_w13, tm_x, di.sms, s)
-                          : moe::launch_gemm(g1, tm_x, tm_w13, di.sms, s));
+    MOE_CUDA_TRY(mx ? (narrow ? moe::launch_gemm_mx_narrow(g1, tm_w13, tm_x, di.sms, s)
+                              : moe::launch_gemm_mx(g1, tm_x, tm_w13, di.sms, s))
+                    : (narrow ? moe::launch_gemm_narrow(g1, tm_w13, tm_x, di.sms, s)
+                              : moe::launch_gemm(g1, tm_x, tm_w13, di.sms, s)));
     MOE_CUDA_TRY(mark(4));
     moe::GemmArgs g2 = g1;
     g2.mode = 1;
@@ -418,9 +418,10 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     g2.act_q = nullptr;
     g2.act_s = nullptr;
     g2.out = static_cast<float*>(at(L.o));
-    MOE_CUDA_TRY(mx       ? moe::launch_gemm_mx(g2, tm_act, tm_w2, di.sms, s)
-                 : narrow ? moe::launch_gemm_narrow(g2, tm_w2, tm_act, di.sms, s)
-                          : moe::launch_gemm(g2, tm_act, tm_w2, di.sms, s));
+    MOE_CUDA_TRY(mx ? (narrow ? moe::launch_gemm_mx_narrow(g2, tm_w2, tm_act, di.sms, s)
+                              : moe::launch_gemm_mx(g2, tm_act, tm_w2, di.sms, s))
+                    : (narrow ? moe::launch_gemm_narrow(g2, tm_w2, tm_act, di.sms, s)
+                              : moe::launch_gemm(g2, tm_act, tm_w2, di.sms, s)));
     MOE_CUDA_TRY(mark(5));
     moe::CombineArgs ca{static_cast<const float*>(at(L.o)), static_cast<const int32_t*>(at(L.row_of)), wts,
                         static_cast<__nv_bfloat16*>(y), T, H, KT, K};

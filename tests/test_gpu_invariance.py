@@ -53,7 +53,7 @@ def test_given_routing_matches_computed():
     assert np.array_equal(y1, y2)
 
 
-@pytest.mark.parametrize("recipe", [0, 1])
+@pytest.mark.parametrize("recipe", [0, 1, 2])
 def test_narrow_and_wide_kernels_agree_bit_for_bit(recipe):
     """A batch with few rows per expert runs the swap-AB (narrow) GEMMs; the same tokens inside a
     large batch run the wide GEMMs.  Both compute each row with the same operations, so the rows
