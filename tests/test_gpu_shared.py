@@ -25,7 +25,11 @@ CASES = {
     "wide_sh": synth.Shape("wide_sh", 300, 256, 256, 2, 2, renormalize=1, biases=True, seed=31,
                            shared_experts=1),                                                   # wide
     "mx_sh": synth.Shape("mx_sh", 96, 256, 384, 8, 2, renormalize=1, recipe=1, biases=True, seed=32,
-                         shared_experts=1),                                                     # MXFP8
+                         shared_experts=1),                                                     # MXFP8, swap-AB
+    "w4_sh": synth.Shape("w4_sh", 96, 256, 384, 8, 2, renormalize=1, recipe=2, biases=True, seed=34,
+                         shared_experts=1),                                                     # W4A8, swap-AB
+    "w4_sh_wide": synth.Shape("w4_sh_wide", 400, 256, 384, 8, 2, renormalize=1, recipe=2, biases=True,
+                              seed=35, shared_experts=1),                                       # W4A8, wide
     "e257_narrow": _E257,                                                                       # 3-kernel permute
     "e257_wide": replace(_E257, name="e257_wide", num_tokens=2048),                             # 3-kernel, wide
 }
@@ -80,7 +84,7 @@ def test_shared_forward_matches_oracle(problems, name):
     assert_y_close(y[tok], r, name)
 
 
-@pytest.mark.parametrize("name", ["tiny_sh", "wide_sh", "mx_sh"])
+@pytest.mark.parametrize("name", ["tiny_sh", "wide_sh", "mx_sh", "w4_sh", "w4_sh_wide"])
 def test_zero_shared_down_projection_keeps_bits(problems, name):
     """Shared expert with w2 = 0 (and no biases): y has the bits of the layer without it."""
     s = replace(CASES[name], biases=False)
