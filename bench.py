@@ -194,6 +194,61 @@ def run_cpu_oracle(shape, prob, n_tokens, threads=None):
     return n_tokens / dt, dt, oracle.num_threads()
 
 
+def gate_only(args, shape, local):
+    """The gate alone (moe_gate: the router matmul on the tensor core, then the RMS-Norm factor and
+    the router top-k) on the problem's hidden states.  Its inputs fit in L2, so L2 is flushed
+    before every launch and each launch is timed by its own CUDA events."""
+    import mixture_experts_fp8_b200 as moe
+
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    x, _, pes = synth.make_activations(shape, device=dev)
+    nw, rw, eps = synth.make_gate(shape, device=dev)
+    cfg = moe.Config(**shape.cfg())
+    gw = moe.transform_gate_weights(cfg, nw, rw)
+    T, H, E, k = shape.num_tokens, shape.hidden, shape.num_experts, shape.top_k
+    lg = torch.empty((T, E), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)      # twice the L2
+    run = lambda: moe.gate(cfg, x, gw, eps, per_expert_scale=pes, logits=lg, topk_idx=idx, topk_weights=w)
+    for _ in range(args.warmup):
+        flush.zero_()
+        run()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    t0 = time.time()
+    for a, b in evs:
+        flush.zero_()
+        a.record()
+        run()
+        b.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    ms = sum(a.elapsed_time(b) for a, b in evs)
+    clocks = sampler.stop((t0, t1))
+    pk, pk_kind = peaks()
+    peak = float(pk["bf16_tflops"])          # burst: each launch is timed alone
+    # three bf16 products per (token, expert, column): the split that keeps fp32 accuracy
+    tc_flops = 3 * 2.0 * T * E * H
+    achieved = tc_flops * args.steps / (ms / 1e3) / 1e12
+    line = {
+        "metric": "gate tokens/s", "value": T * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x3 (fp32-accurate)", "data": "synthetic",
+        "config": {"workload": describe(shape) + "; the gate alone (RMSNorm + router matmul + top-k)",
+                   "l2": "flushed before every launch"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "k_gate_mma + k_route",
+                     "peak_kind": pk_kind + " bf16 burst"},
+        "hbm": {"algorithmic_bytes": 2 * T * H + 6 * E * H + 4 * T * E + 8 * T * k,
+                "GB/s": (2 * T * H + 6 * E * H + 4 * T * E + 8 * T * k) * args.steps / (ms / 1e3) / 1e9},
+        "clocks": clocks, "gpu_launches": 2 * args.steps,
+    }
+    print(json.dumps(line))
+
+
 def reference_arm(args, shape, rank):
     if rank != 0:
         return
@@ -235,6 +290,8 @@ def main():
     ap.add_argument("--gate", action="store_true",
                     help="start each step from the gate (RMSNorm + router matmul + top-k, moe_gate) on "
                          "the bf16 hidden states instead of from precomputed router logits")
+    ap.add_argument("--gate-only", action="store_true",
+                    help="time the gate alone (no expert layer), L2 flushed before every launch")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -253,6 +310,10 @@ def main():
 
     if args.impl == "reference":
         reference_arm(args, shape, rank)
+        return
+    if args.gate_only:
+        if rank == 0:
+            gate_only(args, shape, local)
         return
 
     import mixture_experts_fp8_b200 as moe
@@ -281,6 +342,7 @@ def main():
 
     if args.gate:
         norm_w, router_w, eps = (t.to(dev) if torch.is_tensor(t) else t for t in synth.make_gate(shape))
+        gate_w = moe.transform_gate_weights(cfg, norm_w, router_w)     # once per set of weights
         g_logits = torch.empty((shape.num_tokens, shape.num_experts), dtype=torch.float32, device=dev)
         g_idx = torch.empty((shape.num_tokens, shape.top_k), dtype=torch.int32, device=dev)
         g_w = torch.empty((shape.num_tokens, shape.top_k), dtype=torch.float32, device=dev)
@@ -288,7 +350,7 @@ def main():
     def step(profile=None, x=None):
         x = d.x if x is None else x
         if args.gate:      # the gate replaces the router; the forward takes its routing
-            moe.gate(cfg, x, norm_w, router_w, eps, per_expert_scale=d.per_expert_scale, logits=g_logits,
+            moe.gate(cfg, x, gate_w, eps, per_expert_scale=d.per_expert_scale, logits=g_logits,
                      topk_idx=g_idx, topk_weights=g_w)
             moe.forward(cfg, x, weights, topk_idx=g_idx, topk_weights=g_w, w13_bias=d.w13_bias,
                         w2_bias=d.w2_bias, y=y, expert_counts=counts, workspace=ws, profile=profile)
@@ -358,12 +420,12 @@ def main():
     gate_ms = None
     if args.gate:              # the gate kernel alone, CUDA events on the launch stream
         for _ in range(args.warmup):
-            moe.gate(cfg, d.x, norm_w, router_w, eps, per_expert_scale=d.per_expert_scale, logits=g_logits,
+            moe.gate(cfg, d.x, gate_w, eps, per_expert_scale=d.per_expert_scale, logits=g_logits,
                      topk_idx=g_idx, topk_weights=g_w)
         q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         q0.record()
         for _ in range(args.steps):
-            moe.gate(cfg, d.x, norm_w, router_w, eps, per_expert_scale=d.per_expert_scale, logits=g_logits,
+            moe.gate(cfg, d.x, gate_w, eps, per_expert_scale=d.per_expert_scale, logits=g_logits,
                      topk_idx=g_idx, topk_weights=g_w)
         q1.record()
         torch.cuda.synchronize()
@@ -395,8 +457,8 @@ def main():
         per_step_s = ms / 1e3 / args.steps
         fl = flops(shape, A)
         alg = algorithmic_bytes(shape, active)
-        if args.gate:          # + the router and norm weights (the logits are written instead of read)
-            alg += 4 * shape.num_experts * shape.hidden + 4 * shape.hidden
+        if args.gate:          # + the gate's folded router weights (the logits are written instead of read)
+            alg += 6 * shape.num_experts * shape.hidden
         g1_ms = stage_ms["gemm1_swiglu_requant"] / max(calls, 1)
         g2_ms = stage_ms["gemm2"] / max(calls, 1)
         g1_bytes = gemm1_bytes(shape, active)
@@ -442,9 +504,11 @@ def main():
         }
         if args.gate:
             T, H, E, k = shape.num_tokens, shape.hidden, shape.num_experts, shape.top_k
-            gbytes = 2 * T * H + 4 * H + 4 * E * H + 4 * T * E + 8 * T * k
-            line["gate"] = {"kernel": "k_gate", "ms_per_launch": gate_ms, "algorithmic_bytes": gbytes,
-                            "GB/s": gbytes / (gate_ms / 1e3) / 1e9,
+            # x, the three bf16 parts of the folded router weights, the logits, ids and weights
+            gbytes = 2 * T * H + 6 * E * H + 4 * T * E + 8 * T * k
+            gflops = 2.0 * T * E * H
+            line["gate"] = {"kernel": "k_gate_mma + k_route", "ms_per_launch": gate_ms, "algorithmic_bytes": gbytes,
+                            "GB/s": gbytes / (gate_ms / 1e3) / 1e9, "TFLOP/s": gflops / (gate_ms / 1e3) / 1e12,
                             "note": "stages_ms covers the forward after the gate (its route stage is "
                                     "empty: the routing comes from the gate)"}
         if world == 1 and not args.no_cpu_baseline:

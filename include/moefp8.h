@@ -167,20 +167,34 @@ int moe_route(const moe_config_t *cfg, const float *router_logits, const float *
 /* The gate in front of the router ("mlx_native ops/moe_gate.rs": RMS-Norm of the hidden state,
  * the router matmul, then top-K + softmax + per-expert scale):
  *   logits[t, e] = sum_h ( x[t,h] / sqrt(mean_h x[t,h]^2 + rms_eps) * norm_weight[h] ) * router_weight[e, h]
- * in fp32, computed as r_t * sum_h (x[t,h] * norm_weight[h]) * router_weight[e,h] with the sum in
- * ascending h (a token's logits do not depend on the other tokens or on T), then the router of
- * moe_route on those logits with cfg's routing fields.
- *   hidden_states     device bf16 [T, H], 16-byte aligned
+ * in fp32, computed as r_t * sum_h x[t,h] * w'[e,h] with w'[e,h] = fl32(norm_weight[h] * router_weight[e,h])
+ * and r_t = 1 / sqrt(mean_h x[t,h]^2 + rms_eps), then the router of moe_route on those logits with
+ * cfg's routing fields.
+ *
+ * moe_transform_gate_weights writes w' once per set of weights, as three bf16 parts
+ * hi = rn(w'), mid = rn(w' - hi), lo = rn(w' - hi - mid), each [E, H] row-major, back to back
+ * (moe_gate_weights_size writes 3 * E * H * 2 to *bytes):
  *   norm_weight       device fp32 [H], 16-byte aligned
  *   router_weight     device fp32 [E, H] row-major, 16-byte aligned (E = cfg->num_experts)
+ *   gate_weights      device, moe_gate_weights_size bytes, 16-byte aligned; out
+ *
+ * moe_gate: the sums run on the tensor core (bf16 x times each bf16 part, all accumulated in one
+ * fp32 accumulator, so every product is exact), the H range split in eight fixed shares whose
+ * partial sums are added in share order: a token's logits depend on its own row and on H only,
+ * not on T or on the other tokens.
+ *   hidden_states     device bf16 [T, H], 16-byte aligned
+ *   gate_weights      device, from moe_transform_gate_weights, 16-byte aligned
  *   per_expert_scale  device fp32 [E] or NULL
  *   logits            device fp32 [T, E]  out
  *   topk_idx          device int32 [T, k] out;  topk_weights device fp32 [T, k] out
- * Two launches (the tiled router matmul, then the router).  Feed topk_idx/topk_weights to
- * moe_forward to run the layer on them. */
-int moe_gate(const moe_config_t *cfg, const void *hidden_states, const float *norm_weight,
-             const float *router_weight, float rms_eps, const float *per_expert_scale, float *logits,
-             int32_t *topk_idx, float *topk_weights, void *stream);
+ * Two launches (the router matmul, then the router, which also applies r_t).  A wait that runs
+ * out inside the matmul leaves NaN logits for the tiles it covers.  Feed topk_idx/topk_weights
+ * to moe_forward to run the layer on them. */
+int moe_gate_weights_size(const moe_config_t *cfg, size_t *bytes);
+int moe_transform_gate_weights(const moe_config_t *cfg, const float *norm_weight, const float *router_weight,
+                               void *gate_weights, void *stream);
+int moe_gate(const moe_config_t *cfg, const void *hidden_states, const void *gate_weights, float rms_eps,
+             const float *per_expert_scale, float *logits, int32_t *topk_idx, float *topk_weights, void *stream);
 
 /* The fused layer forward ("MindIE-SD Fused MoE", fused_moe; "MATE Mega MoE",
  * fp8_fp8_mega_moe): route -> permute -> quantize -> gate+up GEMM with SwiGLU and

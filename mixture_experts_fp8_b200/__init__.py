@@ -35,7 +35,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_forward", "moe_forward_profiled",
     "moe_profile_create", "moe_profile_destroy", "moe_profile_read", "moe_profile_reset",
     "moe_read_status", "moe_selftest_bounded_wait", "moe_forward_static_workspace",
-    "moe_debug_inject_fault", "moe_gate",
+    "moe_debug_inject_fault", "moe_gate", "moe_gate_weights_size", "moe_transform_gate_weights",
 )
 MOE_FAULT_NONE = 0
 MOE_FAULT_SKIP_STAGE = 1
@@ -132,7 +132,9 @@ def _load():
             "moe_selftest_bounded_wait": [P, ctypes.c_uint32, P],
             "moe_forward_static_workspace": [CP] + [P] * 13 + [P],
             "moe_debug_inject_fault": [I],
-            "moe_gate": [CP, P, P, P, ctypes.c_float, P, P, P, P, P],
+            "moe_gate": [CP, P, P, ctypes.c_float, P, P, P, P, P],
+            "moe_gate_weights_size": [CP, ctypes.POINTER(S)],
+            "moe_transform_gate_weights": [CP, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -222,9 +224,27 @@ def route(cfg: Config, router_logits, per_expert_scale=None, topk_idx=None, topk
     return topk_idx, topk_weights
 
 
-def gate(cfg: Config, hidden_states, norm_weight, router_weight, rms_eps: float,
-         per_expert_scale=None, logits=None, topk_idx=None, topk_weights=None, stream=None):
-    """RMSNorm + router matmul + router top-k in one launch.
+def gate_weights_size(cfg: Config) -> int:
+    c = cfg.c()
+    n = ctypes.c_size_t()
+    _check(_load().moe_gate_weights_size(ctypes.byref(c), ctypes.byref(n)))
+    return n.value
+
+
+def transform_gate_weights(cfg: Config, norm_weight, router_weight, stream=None):
+    """norm_weight fp32 [H] and router_weight fp32 [E, H] (device) -> the gate's weights: a uint8
+    device tensor holding w' = norm_weight * router_weight as three bf16 parts [3, E, H]."""
+    import torch
+    out = torch.empty(gate_weights_size(cfg), dtype=torch.uint8, device=router_weight.device)
+    c = cfg.c()
+    _check(_load().moe_transform_gate_weights(ctypes.byref(c), _ptr(norm_weight), _ptr(router_weight), _ptr(out),
+                                              _stream(stream)))
+    return out
+
+
+def gate(cfg: Config, hidden_states, gate_weights, rms_eps: float, per_expert_scale=None, logits=None,
+         topk_idx=None, topk_weights=None, stream=None):
+    """RMSNorm + router matmul + router top-k (gate_weights from transform_gate_weights).
     -> (logits fp32 [T, E], topk_idx int32 [T, k], topk_weights fp32 [T, k])."""
     import torch
     T, E, k = cfg.num_tokens, cfg.num_experts, cfg.top_k
@@ -236,9 +256,9 @@ def gate(cfg: Config, hidden_states, norm_weight, router_weight, rms_eps: float,
     if topk_weights is None:
         topk_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
     c = cfg.c()
-    _check(_load().moe_gate(ctypes.byref(c), _ptr(hidden_states), _ptr(norm_weight), _ptr(router_weight),
-                            ctypes.c_float(rms_eps), _ptr(per_expert_scale), _ptr(logits), _ptr(topk_idx),
-                            _ptr(topk_weights), _stream(stream)))
+    _check(_load().moe_gate(ctypes.byref(c), _ptr(hidden_states), _ptr(gate_weights), ctypes.c_float(rms_eps),
+                            _ptr(per_expert_scale), _ptr(logits), _ptr(topk_idx), _ptr(topk_weights),
+                            _stream(stream)))
     return logits, topk_idx, topk_weights
 
 

@@ -34,14 +34,18 @@ struct RouteArgs {
     int T, E, K, routing, renorm, G, kg, mode;
     float rsf;
     int32_t* status;            // cleared to MOE_OK by the first thread when non-null
+    // Gate mode (moe_gate): when gate_x is set, logits holds the router matmul's sums
+    // sum_h x[t,h] * w'[e,h]; each token's row is first scaled in place by its RMS-Norm factor
+    // 1 / sqrt(mean_h x[t,h]^2 + gate_eps), then routed.
+    const __nv_bfloat16* gate_x = nullptr;   // [T, gate_H]
+    int gate_H = 0;
+    float gate_eps = 0.0f;
 };
 
+// The gate's router matmul (k_gate_mma): logits[t, e] = sum_h x[t,h] * w'[e,h] from the tensor
+// maps of x and of the three bf16 parts of w'.
 struct GateArgs {
-    const __nv_bfloat16* x;     // [T, H]
-    const float* norm_w;        // [H]
-    const float* router_w;      // [E, H]
     float* logits;              // [T, E] out
-    float eps;
     int T, H, E;
 };
 
@@ -110,8 +114,12 @@ struct GemmArgs {
 };
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
-cudaError_t launch_gate(const GateArgs& g, const RouteArgs& ra, cudaStream_t s);
-size_t gate_smem_bytes(int H);
+cudaError_t launch_gate(const CUtensorMap& tmX, const CUtensorMap& tmW, const GateArgs& g, const RouteArgs& ra,
+                        cudaStream_t s);
+cudaError_t launch_gate_split(const float* norm_w, const float* router_w, void* out, int E, int H, cudaStream_t s);
+// Rows of the tensor-map boxes k_gate_mma expects: tokens (x) and experts (w' parts).
+uint32_t gate_token_box();
+uint32_t gate_weight_box();
 cudaError_t launch_permute(const PermuteArgs& a, cudaStream_t s);
 cudaError_t launch_permute_small(const PermuteArgs& pa, bool clear_status, cudaStream_t s);
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s);

@@ -430,27 +430,54 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
     return ok();
 }
 
-int moe_gate(const moe_config_t* cfg, const void* hidden_states, const float* norm_weight,
-             const float* router_weight, float rms_eps, const float* per_expert_scale, float* logits,
-             int32_t* topk_idx, float* topk_weights, void* stream) {
+int moe_gate_weights_size(const moe_config_t* cfg, size_t* bytes) {
     int rc = check_config(cfg);
     if (rc) return rc;
-    if (!hidden_states || !norm_weight || !router_weight || !logits || !topk_idx || !topk_weights)
+    if (!bytes) return fail(MOE_ERR_INVALID_ARG, "moe_gate_weights_size: NULL output");
+    *bytes = static_cast<size_t>(3) * cfg->num_experts * cfg->hidden * 2;
+    return ok();
+}
+
+int moe_transform_gate_weights(const moe_config_t* cfg, const float* norm_weight, const float* router_weight,
+                               void* gate_weights, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!norm_weight || !router_weight || !gate_weights)
+        return fail(MOE_ERR_INVALID_ARG, "moe_transform_gate_weights: NULL pointer");
+    if (!aligned(norm_weight, 16) || !aligned(router_weight, 16) || !aligned(gate_weights, 16))
+        return fail(MOE_ERR_INVALID_ARG, "moe_transform_gate_weights: buffers need 16-byte alignment");
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    MOE_CUDA_TRY(moe::launch_gate_split(norm_weight, router_weight, gate_weights, cfg->num_experts, cfg->hidden,
+                                        static_cast<cudaStream_t>(stream)));
+    return ok();
+}
+
+int moe_gate(const moe_config_t* cfg, const void* hidden_states, const void* gate_weights, float rms_eps,
+             const float* per_expert_scale, float* logits, int32_t* topk_idx, float* topk_weights, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!hidden_states || !gate_weights || !logits || !topk_idx || !topk_weights)
         return fail(MOE_ERR_INVALID_ARG, "moe_gate: NULL pointer");
-    if (!aligned(hidden_states, 16) || !aligned(router_weight, 16) || !aligned(norm_weight, 16) ||
-        !aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_weights, 4) ||
-        (per_expert_scale && !aligned(per_expert_scale, 4)))
-        return fail(MOE_ERR_INVALID_ARG,
-                    "moe_gate: misaligned buffer (hidden_states, norm_weight and router_weight need 16 bytes)");
+    if (!aligned(hidden_states, 16) || !aligned(gate_weights, 16) || !aligned(logits, 4) || !aligned(topk_idx, 4) ||
+        !aligned(topk_weights, 4) || (per_expert_scale && !aligned(per_expert_scale, 4)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_gate: misaligned buffer (hidden_states and gate_weights need 16 bytes)");
     if (!(rms_eps >= 0.0f)) return fail(MOE_ERR_INVALID_ARG, "moe_gate: rms_eps must be >= 0");
     DeviceInfo di;
     if ((rc = device_info(&di))) return rc;
-    moe::GateArgs g{static_cast<const __nv_bfloat16*>(hidden_states), norm_weight, router_weight, logits, rms_eps,
-                    cfg->num_tokens, cfg->hidden, cfg->num_experts};
-    moe::RouteArgs ra{logits, per_expert_scale, topk_idx, topk_weights, cfg->num_tokens, cfg->num_experts,
-                      cfg->top_k, cfg->routing, cfg->renormalize, cfg->group_count, cfg->k_group,
-                      cfg->group_select_mode, cfg->routed_scaling_factor, nullptr};
-    MOE_CUDA_TRY(moe::launch_gate(g, ra, static_cast<cudaStream_t>(stream)));
+    const int T = cfg->num_tokens, H = cfg->hidden, E = cfg->num_experts;
+    // bf16 rows viewed as bytes: 64 columns = one 128-byte box row
+    CUtensorMap tm_x, tm_w;
+    if ((rc = make_kmajor_map(&tm_x, hidden_states, T, 2ull * H, moe::gate_token_box()))) return rc;
+    if ((rc = make_kmajor_map(&tm_w, gate_weights, 3ull * E, 2ull * H, moe::gate_weight_box()))) return rc;
+    moe::GateArgs g{logits, T, H, E};
+    moe::RouteArgs ra{logits, per_expert_scale, topk_idx, topk_weights, T, E, cfg->top_k, cfg->routing,
+                      cfg->renormalize, cfg->group_count, cfg->k_group, cfg->group_select_mode,
+                      cfg->routed_scaling_factor, nullptr};
+    ra.gate_x = static_cast<const __nv_bfloat16*>(hidden_states);
+    ra.gate_H = H;
+    ra.gate_eps = rms_eps;
+    MOE_CUDA_TRY(moe::launch_gate(tm_x, tm_w, g, ra, static_cast<cudaStream_t>(stream)));
     return ok();
 }
 
