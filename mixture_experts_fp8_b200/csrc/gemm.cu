@@ -153,6 +153,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmB);
     }
     if (warp == 1) tmem_alloc(tmem_holder, kTmemCols);
+    if (warp == 0) {   // the first unit's weight tiles toward L2 while the preceding kernel runs
+        int e, nb;
+        if (early_unit_tiles(p.tile_start, p.E, nt, blockIdx.x, lane, e, nb) && lane == 0)
+            prefetch_weight_stages(&tmB, e * p.N + nb * kTileN, p.K);
+    }
     // everything above overlaps the previous kernel; its outputs are read only from here on
     pdl_wait_then_release();
     for (int i = threadIdx.x; i <= p.E; i += kThreads) {

@@ -18,6 +18,68 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// ------------------------------------------------------------------ weight prefetch before the wait
+// Before its wait on the preceding kernel, a GEMM CTA hints the weight tiles of its first work
+// unit into L2: the weights do not come from that kernel, so their fetch can overlap it.  The
+// unit's expert is found from the permutation's outputs (offsets, tile_start), read from L2 by
+// one warp.  The permutation completed before the preceding kernel started its work, and a stale
+// value could only make the hint miss: the real loads use the values read after the wait.
+constexpr int kPrefetchStages = 6;
+
+// Narrow kernels: expert e owns nblk * ceil(rows_e / NT) units, weight block by weight block
+// (a warp scan of the per-expert unit counts).
+template <int NT>
+__device__ __forceinline__ bool early_unit_rows(const int* offsets, int E, int nblk, int u, int lane, int& e_out,
+                                                int& blk_out) {
+    int base = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        int n = 0;
+        if (e < E) n = nblk * ((__ldcg(offsets + e + 1) - __ldcg(offsets + e) + NT - 1) / NT);
+        int incl = n;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const int excl = base + incl - n;
+        const unsigned m = __ballot_sync(0xffffffffu, n > 0 && u >= excl && u < excl + n);
+        if (m) {
+            const int src = __ffs(m) - 1;
+            const int ex = __shfl_sync(0xffffffffu, excl, src), nn = __shfl_sync(0xffffffffu, n, src);
+            e_out = e0 + src;
+            blk_out = (u - ex) / (nn / nblk);
+            return true;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return false;
+}
+
+// Wide kernels: expert e owns units [nt * tile_start[e], nt * tile_start[e+1]), column block by
+// column block; the expert is the last one whose first unit is <= u.
+__device__ __forceinline__ bool early_unit_tiles(const int* tile_start, int E, int nt, int u, int lane, int& e_out,
+                                                 int& blk_out) {
+    if (u >= nt * __ldcg(tile_start + E)) return false;
+    int cnt = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        cnt += __popc(__ballot_sync(0xffffffffu, e < E && nt * __ldcg(tile_start + e) <= u));
+    }
+    const int e = cnt - 1;
+    const int t0 = __ldcg(tile_start + e), mt = __ldcg(tile_start + e + 1) - t0;
+    if (e < 0 || mt <= 0) return false;
+    e_out = e;
+    blk_out = (u - nt * t0) / mt;
+    return true;
+}
+
+// One thread: the first n K stages of the weight box at row `row` toward L2.
+__device__ __forceinline__ void prefetch_weight_stages(const CUtensorMap* map, int row, int K) {
+    const int n = min(kPrefetchStages, K / kTileK);
+    for (int kb = 0; kb < n; ++kb) tma_prefetch_2d(map, kb * kTileK, row);
+}
+
 // Poll intervals of the single-thread roles, which mostly wait on the epilogue warps (the
 // producer for a free stage, the MMA issuer for a free accumulator): sleeping between polls keeps
 // them from taking issue slots on the schedulers they share with epilogue warps.

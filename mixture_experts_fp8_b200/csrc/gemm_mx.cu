@@ -112,6 +112,11 @@ __global__ void __launch_bounds__(kXThreads, 1)
         prefetch_tmap(&tmB);
     }
     if (warp == 1) tmem_alloc(tmem_holder, kXTmemCols);
+    if (warp == 0) {   // the first unit's weight tiles toward L2 while the preceding kernel runs
+        int e, nb;
+        if (early_unit_tiles(p.tile_start, p.E, nt, blockIdx.x, lane, e, nb) && lane == 0)
+            prefetch_weight_stages(&tmB, e * p.N + nb * kXN, p.K);
+    }
     pdl_wait_then_release();
     for (int i = threadIdx.x; i <= p.E; i += kXThreads) {
         s_tstart[i] = p.tile_start[i];

@@ -123,6 +123,11 @@ __global__ void __launch_bounds__(kQThreads, 1)
         prefetch_tmap(&tmT);
     }
     if (warp == 1) tmem_alloc(tmem_holder, kQTmemCols);
+    if (warp == 0) {   // the first unit's weight tiles toward L2 while the preceding kernel runs
+        int e, nb;
+        if (early_unit_rows<kQT>(p.offsets, p.E, nt, blockIdx.x, lane, e, nb) && lane == 0)
+            prefetch_weight_stages(&tmW, e * p.N + nb * kTileM, p.K);
+    }
     pdl_wait_then_release();
     for (int i = threadIdx.x; i <= p.E; i += kQThreads) s_off[i] = p.offsets[i];
     __syncthreads();

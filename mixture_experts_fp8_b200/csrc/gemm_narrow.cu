@@ -121,6 +121,11 @@ __global__ void __launch_bounds__(kNThreads, 1)
         prefetch_tmap(&tmT);
     }
     if (warp == 1) tmem_alloc(tmem_holder, kNTmemCols);
+    if (warp == 0) {   // the first unit's weight tiles toward L2 while the preceding kernel runs
+        int e, wb;
+        if (early_unit_rows<kNT>(p.offsets, p.E, nwb, blockIdx.x, lane, e, wb) && lane == 0)
+            prefetch_weight_stages(&tmW, e * p.N + wb * 256, p.K);
+    }
     pdl_wait_then_release();
     for (int i = threadIdx.x; i <= p.E; i += kNThreads) s_off[i] = p.offsets[i];
     __syncthreads();
