@@ -194,6 +194,21 @@ def run_cpu_oracle(shape, prob, n_tokens, threads=None):
     return n_tokens / dt, dt, oracle.num_threads()
 
 
+def reduce_max(value: float, dist=None, device="cpu") -> float:
+    """The largest of the ranks' values, returned on every rank (one all-reduce; the identity
+    without a process group).  Multi-GPU times are the slowest rank's."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_rank: int, steps: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_max / 1e3)
+
+
 def gate_only(args, shape, local):
     """The gate alone (moe_gate: the router matmul on the tensor core, then the RMS-Norm factor and
     the router top-k) on the problem's hidden states.  Its inputs fit in L2, so L2 is flushed
@@ -384,10 +399,7 @@ def main():
         dist.barrier()
     ms = start.elapsed_time(end)
     clocks = sampler.stop((t_wall0, t_wall1))
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(ms, dist, dev)
     # per-stage device times: K more forwards with CUDA events recorded by the library between the
     # stages, on the launch stream
     prof = moe.Profile()
@@ -443,17 +455,15 @@ def main():
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = reduce_max(e2e_ms, dist, dev)
     if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
 
     if rank == 0:
         pk, pk_kind = peaks()
         hbm = float(pk["hbm_gbs"])
         fp8_peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])) * FP8_OVER_BF16
-        tok_s = world * shape.num_tokens * args.steps / (ms / 1e3)
+        tok_s = job_tokens_per_s(world, shape.num_tokens, args.steps, ms)
         per_step_s = ms / 1e3 / args.steps
         fl = flops(shape, A)
         alg = algorithmic_bytes(shape, active)
