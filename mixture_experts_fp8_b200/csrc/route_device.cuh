@@ -1,5 +1,5 @@
-// route_device.cuh -- per-token router top-k, one warp per token (shared by the router kernel and
-// the fused small-batch route + permute kernel).
+// route_device.cuh -- per-token router top-k, one warp per token (the body of the router kernel,
+// k_route, for moe_route, the forward and the gate).
 //
 // "MindIE-SD Fused MoE", routing selection and parameter table: softmax or sigmoid scores,
 // optional expert-group pre-selection (group score = max, or sum of the two largest), top_k
