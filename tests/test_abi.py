@@ -124,3 +124,25 @@ def test_interleave_is_a_permutation():
         assert sorted(rows) == list(range(2 * I))
         for i in range(I):
             assert rows[I + i] - rows[i] == blk
+
+def test_gate_entry_points_validate_before_any_cuda_call():
+    """moe_gate_weights_size reports 3 bf16 parts of [E, H]; the gate's transform and call reject
+    NULL and misaligned buffers and a negative epsilon with a message, touching no device."""
+    lib = moe.lib()
+    c = cfg(num_experts=24, hidden=384, top_k=3)
+    assert moe.gate_weights_size(c) == 3 * 24 * 384 * 2
+    cc = c.c()
+    rc = lib.moe_transform_gate_weights(ctypes.byref(cc), None, None, None, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"NULL" in lib.moe_last_error()
+    buf = ctypes.create_string_buffer(64)
+    odd = ctypes.addressof(buf) | 4                 # 4-byte aligned, not 16
+    rc = lib.moe_transform_gate_weights(ctypes.byref(cc), odd, odd, odd, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"16-byte" in lib.moe_last_error()
+    rc = lib.moe_gate(ctypes.byref(cc), None, None, ctypes.c_float(1e-6), None, None, None, None, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"NULL" in lib.moe_last_error()
+    al = (ctypes.addressof(buf) + 15) & ~15
+    rc = lib.moe_gate(ctypes.byref(cc), al, al, ctypes.c_float(-1.0), None, al, al, al, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"rms_eps" in lib.moe_last_error()
+    bad = moe.Config(num_tokens=0, hidden=384, inter=128, num_experts=24, top_k=3).c()
+    n = ctypes.c_size_t(0)
+    assert lib.moe_gate_weights_size(ctypes.byref(bad), ctypes.byref(n)) == moe.MOE_ERR_INVALID_ARG
