@@ -268,7 +268,9 @@ def reference_arm(args, shape, rank):
     if rank != 0:
         return
     prob = synth.make_problem(shape, device="cpu")
-    n = {"tiny": 16, "decode": 8, "skewed": 16, "prefill": 2, "large": 4}.get(shape.name, 4)
+    # tokens per step: the whole batch where one oracle call on it takes well under a second
+    # (tiny, decode), else a sample sized so that a step stays near a second
+    n = {"tiny": 16, "decode": 64, "decode_w4a8": 64, "skewed": 16, "prefill": 2, "large": 4}.get(shape.name, 4)
     for _ in range(args.warmup):
         run_cpu_oracle(shape, prob, 1)
     times = []
