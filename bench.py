@@ -307,6 +307,8 @@ def main():
     ap.add_argument("--gate", action="store_true",
                     help="start each step from the gate (RMSNorm + router matmul + top-k, moe_gate) on "
                          "the bf16 hidden states instead of from precomputed router logits")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every kernel from the host instead of replaying a captured CUDA graph")
     ap.add_argument("--gate-only", action="store_true",
                     help="time the gate alone (no expert layer), L2 flushed before every launch")
     args = ap.parse_args()
@@ -383,6 +385,30 @@ def main():
     active = int((counts.cpu() > 0).sum())
     A = shape.num_tokens * (shape.top_k + shape.shared_experts)   # rows through the GEMMs
 
+    # Several consecutive steps captured into one CUDA graph: a replay is one host call instead of
+    # six to eight launches per step, and inside the graph each step's first kernel still overlaps
+    # the previous step's last one (programmatic dependent launch edges).  Eager launches with
+    # --no-graph, or when the capture fails (reported in the line).
+    run, per_run = step, 1
+    graph_info = {"used": False, "why": "--no-graph"}
+    if not args.no_graph:
+        try:
+            gs = next(n for n in (10, 8, 5, 4, 2, 1) if args.steps % n == 0)
+            y_eager = y.clone()
+            g_step = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_step):
+                for _ in range(gs):
+                    step()
+            y.zero_()
+            g_step.replay()
+            torch.cuda.synchronize()
+            run, per_run = g_step.replay, gs
+            graph_info = {"used": True, "steps_per_graph": gs,
+                          "same_output_as_eager": bool(torch.equal(y, y_eager))}
+        except Exception as exc:   # noqa: BLE001 - any capture failure falls back to launches
+            torch.cuda.synchronize()
+            graph_info = {"used": False, "why": f"capture failed: {exc}"[:300]}
+
     # timed region: K plain forwards (no events between the kernels, which would break their
     # programmatic-dependent-launch overlap)
     sampler = ClockSampler(local)
@@ -392,8 +418,8 @@ def main():
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start.record()
-    for _ in range(args.steps):
-        step()
+    for _ in range(args.steps // per_run):
+        run()
     end.record()
     torch.cuda.synchronize()
     t_wall1 = time.time()
@@ -442,6 +468,19 @@ def main():
             moe.forward(cfg, x_in, weights, router_logits=l_in, per_expert_scale=d.per_expert_scale,
                         w13_bias=d.w13_bias, w2_bias=d.w2_bias, y=y_out, workspace=ws)
 
+    e2e_graphs = None
+    if graph_info["used"]:     # one graph per buffer slot
+        try:
+            e2e_graphs = []
+            for b in range(NB):
+                gg = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gg):
+                    fwd(x_d[b], l_d[b], y_d[b])
+                e2e_graphs.append(gg)
+        except Exception:          # noqa: BLE001
+            torch.cuda.synchronize()
+            e2e_graphs = None
+
     def e2e_step(i):
         b = i % NB
         with torch.cuda.stream(s_in):
@@ -454,7 +493,10 @@ def main():
         s_c.wait_event(in_done[b])
         if used[b]:
             s_c.wait_event(out_done[b])               # slot b's previous result has left
-        fwd(x_d[b], l_d[b], y_d[b])
+        if e2e_graphs:
+            e2e_graphs[b].replay()
+        else:
+            fwd(x_d[b], l_d[b], y_d[b])
         fwd_done[b].record(s_c)
         with torch.cuda.stream(s_out):
             s_out.wait_event(fwd_done[b])
@@ -546,6 +588,7 @@ def main():
             "ms_per_step_with_stage_events": ms_profiled / args.steps,
             "gemm2": {"ms": g2_ms, "GB/s": gemm2_bytes(shape, active) / (g2_ms / 1e3) / 1e9},
             "clocks": clocks, "gpu_launches": kernels_per_step(A) * args.steps, "status": status,
+            "graph": dict(graph_info, e2e=e2e_graphs is not None),
             "e2e": {"value": world * shape.num_tokens * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": x_h.numel() * 2 + (0 if args.gate else l_h.numel() * 4),
                     "d2h_bytes_per_step": y_h[0].numel() * 2,
