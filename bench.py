@@ -389,22 +389,36 @@ def main():
     # six to eight launches per step, and inside the graph each step's first kernel still overlaps
     # the previous step's last one (programmatic dependent launch edges).  Eager launches with
     # --no-graph, or when the capture fails (reported in the line).
-    run, per_run = step, 1
+    def capture(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(n):
+                step()
+        return g
+
+    def timed_steps():             # exactly args.steps steps
+        for _ in range(args.steps):
+            step()
+
+    run = timed_steps
     graph_info = {"used": False, "why": "--no-graph"}
     if not args.no_graph:
         try:
-            gs = next(n for n in (10, 8, 5, 4, 2, 1) if args.steps % n == 0)
+            gs = 10
             y_eager = y.clone()
-            g_step = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_step):
-                for _ in range(gs):
-                    step()
+            g_main = capture(gs)
+            g_rest = capture(args.steps % gs) if args.steps % gs else None
             y.zero_()
-            g_step.replay()
+            g_main.replay()
             torch.cuda.synchronize()
-            run, per_run = g_step.replay, gs
-            graph_info = {"used": True, "steps_per_graph": gs,
-                          "same_output_as_eager": bool(torch.equal(y, y_eager))}
+            same = bool(torch.equal(y, y_eager))
+
+            def run():
+                for _ in range(args.steps // gs):
+                    g_main.replay()
+                if g_rest is not None:
+                    g_rest.replay()
+            graph_info = {"used": True, "steps_per_graph": gs, "same_output_as_eager": same}
         except Exception as exc:   # noqa: BLE001 - any capture failure falls back to launches
             torch.cuda.synchronize()
             graph_info = {"used": False, "why": f"capture failed: {exc}"[:300]}
@@ -418,8 +432,7 @@ def main():
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start.record()
-    for _ in range(args.steps // per_run):
-        run()
+    run()
     end.record()
     torch.cuda.synchronize()
     t_wall1 = time.time()
