@@ -1,13 +1,18 @@
 """Benchmark of the fused FP8 routed-expert MoE layer forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode|tiny|prefill|skewed|large]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--config decode|tiny|prefill|skewed|large|decode_w4a8|prefill_w4a8]
                     [--impl reference] [--no-cpu-baseline] [--tokens T] [--shared-expert]
+                    [--recipe 0|1|2] [--gate | --gate-only] [--no-graph]
 
 One step = one moe_forward call (route, permute, quantize, gate+up GEMM with SwiGLU and
 requantization, down GEMM, combine) over one batch of seeded synthetic inputs of the named
 problem, inputs resident in HBM.  The default problem is the decode configuration (64 tokens,
 H 2816, I 768, 128 experts, top-8); its ~0.85 GB of FP8 weights exceed the 126 MB L2, so every
-step streams them from HBM.
+step streams them from HBM.  The timed loop replays a CUDA graph of 10 steps (--no-graph:
+host launches); the e2e figure copies each step's inputs in and its output out through pinned
+host memory, on copy streams that overlap the neighbouring steps.  --gate starts every step from
+the gate (moe_gate) instead of router logits; --gate-only times the gate alone.
 
 Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) are independent replicas, one per
 GPU, with no collective on the data path ("scaling": "weak"); timing is the max over ranks.
