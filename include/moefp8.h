@@ -258,6 +258,54 @@ int moe_forward_profiled(const moe_config_t *cfg, const void *hidden_states,
                          int32_t *expert_counts, void *workspace, size_t workspace_bytes,
                          moe_profile_t *prof, void *stream);
 
+/* Expert parallelism over `ranks` ranks of one node ("MindIE-SD Fused MoE", execution flow:
+ * dispatch, mlp, combine, and the dynamic dispatcher's all-to-all; "MATE Mega MoE", Typical
+ * Flow: up to 8 intranode ranks).  Rank r owns experts r*E/R .. (r+1)*E/R - 1 (E % R == 0, no
+ * shared expert); each rank routes its own T tokens with moe_route, then:
+ *
+ * moe_ep_dispatch orders this rank's A = T*k routed slots (slot = t*k + j) by destination rank,
+ * stable in slot order, and gathers what each destination needs.  cfg: this rank's tokens, the
+ * global expert count.
+ *   hidden_states   device bf16 [T, H], 16-byte aligned
+ *   topk_idx        device int32 [T, k]: global expert ids
+ *   send_counts     device int32 [ranks]   out: slots going to each rank
+ *   send_x          device bf16 [A, H]     out: each slot's token row, in send order (16-byte aligned)
+ *   send_expert     device int32 [A]       out: each slot's expert id local to its destination
+ *   slot_pos        device int32 [T, k]    out: each slot's position in send order
+ *   workspace       as for moe_forward with the same cfg (scratch for the ordering)
+ *   Four launches.  An expert id outside [0, E) is reported as MOE_ERR_BOUNDS in the workspace's
+ *   status word (moe_read_status) and its slot is not sent.
+ *
+ * The caller then exchanges send_x and send_expert (all-to-all with the counts: NCCL, or peer
+ * copies), and every rank runs moe_forward_rows on the N rows it received:
+ *
+ * moe_forward_rows: each row through one local expert with weight 1.  cfg: num_tokens = N,
+ * top_k = 1, num_experts = E/R, no shared expert; weights from moe_transform_weights on this
+ * rank's experts.
+ *   rows            device bf16 [N, H], 16-byte aligned
+ *   expert_of_row   device int32 [N]: local expert ids
+ *   o_rows          device fp32 [N, H] out, 16-byte aligned: each row's GEMM2 output (+ b2), in row
+ *                   order, bit-identical to the same row's output inside moe_forward (a row's
+ *                   result depends only on its own codes and its expert's weights)
+ *   The forward's launches, the last one copying the rows out in row order.
+ *
+ * The caller returns the rows (the reverse all-to-all), so that o_home[i] belongs to send
+ * position i, and combines them on the home rank:
+ *
+ * moe_combine_rows: y[t] = bf16_rn( sum_j topk_weights[t,j] * o_home[slot_pos[t,j]] ), fp32, in
+ * slot order: the combine of moe_forward, so y is bit-identical to the single-GPU forward.
+ *   o_rows          device fp32 [T*k, H], 16-byte aligned;  y device bf16 [T, H], 16-byte aligned
+ *   One launch. */
+int moe_ep_dispatch(const moe_config_t *cfg, int ranks, const void *hidden_states, const int32_t *topk_idx,
+                    int32_t *send_counts, void *send_x, int32_t *send_expert, int32_t *slot_pos,
+                    void *workspace, size_t workspace_bytes, void *stream);
+int moe_forward_rows(const moe_config_t *cfg, const void *rows, const int32_t *expert_of_row,
+                     const void *w13_t, const void *w13s_t, const void *w2_t, const void *w2s_t,
+                     const void *w13_bias, const void *w2_bias, float *o_rows, void *workspace,
+                     size_t workspace_bytes, void *stream);
+int moe_combine_rows(const moe_config_t *cfg, const float *o_rows, const int32_t *slot_pos,
+                     const float *topk_weights, void *y, void *stream);
+
 /* Create / destroy a stage profiler (creates CUDA events on the current device). */
 int moe_profile_create(moe_profile_t **prof);
 int moe_profile_destroy(moe_profile_t *prof);

@@ -36,6 +36,7 @@ EXPORTED = (
     "moe_profile_create", "moe_profile_destroy", "moe_profile_read", "moe_profile_reset",
     "moe_read_status", "moe_selftest_bounded_wait", "moe_forward_static_workspace",
     "moe_debug_inject_fault", "moe_gate", "moe_gate_weights_size", "moe_transform_gate_weights",
+    "moe_ep_dispatch", "moe_forward_rows", "moe_combine_rows",
 )
 MOE_FAULT_NONE = 0
 MOE_FAULT_SKIP_STAGE = 1
@@ -135,6 +136,9 @@ def _load():
             "moe_gate": [CP, P, P, ctypes.c_float, P, P, P, P, P],
             "moe_gate_weights_size": [CP, ctypes.POINTER(S)],
             "moe_transform_gate_weights": [CP, P, P, P, P],
+            "moe_ep_dispatch": [CP, I, P, P, P, P, P, P, P, S, P],
+            "moe_forward_rows": [CP] + [P] * 10 + [S, P],
+            "moe_combine_rows": [CP, P, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -260,6 +264,53 @@ def gate(cfg: Config, hidden_states, gate_weights, rms_eps: float, per_expert_sc
                             _ptr(per_expert_scale), _ptr(logits), _ptr(topk_idx), _ptr(topk_weights),
                             _stream(stream)))
     return logits, topk_idx, topk_weights
+
+
+def ep_dispatch(cfg: Config, ranks: int, hidden_states, topk_idx, workspace, stream=None):
+    """Order this rank's routed slots by destination rank (rank r owns experts r*E/R ..) ->
+    (send_counts int32 [R], send_x bf16 [T*k, H], send_expert int32 [T*k], slot_pos int32 [T, k])."""
+    import torch
+    T, H, k = cfg.num_tokens, cfg.hidden, cfg.top_k
+    dev = hidden_states.device
+    send_counts = torch.empty(ranks, dtype=torch.int32, device=dev)
+    send_x = torch.empty((T * k, H), dtype=torch.bfloat16, device=dev)
+    send_expert = torch.empty(T * k, dtype=torch.int32, device=dev)
+    slot_pos = torch.empty((T, k), dtype=torch.int32, device=dev)
+    c = cfg.c()
+    _check(_load().moe_ep_dispatch(ctypes.byref(c), int(ranks), _ptr(hidden_states), _ptr(topk_idx),
+                                   _ptr(send_counts), _ptr(send_x), _ptr(send_expert), _ptr(slot_pos),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)))
+    return send_counts, send_x, send_expert, slot_pos
+
+
+def forward_rows(cfg: Config, rows, expert_of_row, weights, w13_bias=None, w2_bias=None, o_rows=None,
+                 workspace=None, stream=None):
+    """Each row through one local expert with weight 1 (cfg: num_tokens = rows, top_k = 1,
+    num_experts = this rank's experts) -> o_rows fp32 [N, H]."""
+    import torch
+    N, H = cfg.num_tokens, cfg.hidden
+    if o_rows is None:
+        o_rows = torch.empty((N, H), dtype=torch.float32, device=rows.device)
+    if workspace is None:
+        workspace = new_workspace(cfg, rows.device)
+    c = cfg.c()
+    w13_t, w13s_t, w2_t, w2s_t = weights
+    _check(_load().moe_forward_rows(ctypes.byref(c), _ptr(rows), _ptr(expert_of_row), _ptr(w13_t), _ptr(w13s_t),
+                                    _ptr(w2_t), _ptr(w2s_t), _ptr(w13_bias), _ptr(w2_bias), _ptr(o_rows),
+                                    _ptr(workspace), workspace.numel(), _stream(stream)))
+    return o_rows
+
+
+def combine_rows(cfg: Config, o_rows, slot_pos, topk_weights, y=None, stream=None):
+    """y[t] = bf16(sum_j w[t,j] * o_rows[slot_pos[t,j]]) in slot order -> y bf16 [T, H]."""
+    import torch
+    T, H = cfg.num_tokens, cfg.hidden
+    if y is None:
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=o_rows.device)
+    c = cfg.c()
+    _check(_load().moe_combine_rows(ctypes.byref(c), _ptr(o_rows), _ptr(slot_pos), _ptr(topk_weights), _ptr(y),
+                                    _stream(stream)))
+    return y
 
 
 def forward(cfg: Config, hidden_states, weights, router_logits=None, per_expert_scale=None,

@@ -90,6 +90,18 @@ struct CombineArgs {
     int T, H, K, k;             // slots j >= k (the shared expert's) have weight 1
 };
 
+// Expert parallelism (ep.cu): slot i = t * K + j of this rank's routing.
+struct EpArgs {
+    const int32_t* idx;           // [A] routed expert ids (global numbering)
+    int32_t* dest;                // [A] out (k_ep_dest): destination rank, -1 for an invalid id
+    const int32_t* row_src;       // [A] send order -> slot (from the permutation by destination)
+    const __nv_bfloat16* x;       // [T, H] this rank's tokens
+    __nv_bfloat16* send_x;        // [A, H] out: token rows in send order
+    int32_t* send_expert;         // [A] out: expert id local to the destination rank
+    int32_t* status;
+    int A, K, H, E, e_loc;        // e_loc = E / ranks
+};
+
 struct TransformArgs {
     const uint8_t* w13; const void* w13s; const uint8_t* w2; const void* w2s;
     uint8_t* w13_t; void* w13s_t; uint8_t* w2_t; void* w2s_t;
@@ -125,6 +137,10 @@ cudaError_t launch_permute_small(const PermuteArgs& pa, bool clear_status, cudaS
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_transform(const TransformArgs& a, cudaStream_t s);
+cudaError_t launch_ep_dest(const EpArgs& a, cudaStream_t s);
+cudaError_t launch_ep_gather(const EpArgs& a, cudaStream_t s);
+cudaError_t launch_rows_f32(const float* o, const int32_t* row_of, float* out, int T, int H, int32_t* status,
+                            cudaStream_t s);
 // Rows of the weight tensor-map box the wide kernel expects for each mode.
 uint32_t gemm_weight_box(int mode);
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB,

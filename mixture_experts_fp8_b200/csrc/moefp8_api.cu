@@ -301,19 +301,25 @@ int moe_route(const moe_config_t* cfg, const float* router_logits, const float* 
     return ok();
 }
 
-int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, const float* router_logits,
-                         const float* per_expert_scale, const int32_t* topk_idx, const float* topk_weights,
-                         const void* w13_t, const void* w13s_t, const void* w2_t, const void* w2s_t,
-                         const void* w13_bias, const void* w2_bias, void* y, int32_t* expert_counts, void* workspace,
-                         size_t workspace_bytes, moe_profile_t* prof, void* stream_) {
+namespace {
+
+// The forward.  Its last stage is the combine into bf16 y, or, with o_rows set (one slot per row,
+// the expert side of expert parallelism), the fp32 GEMM2 rows copied out in row order.
+int forward_impl(const moe_config_t* cfg, const void* hidden_states, const float* router_logits,
+                 const float* per_expert_scale, const int32_t* topk_idx, const float* topk_weights,
+                 const void* w13_t, const void* w13s_t, const void* w2_t, const void* w2s_t,
+                 const void* w13_bias, const void* w2_bias, void* y, float* o_rows, int32_t* expert_counts,
+                 void* workspace, size_t workspace_bytes, moe_profile_t* prof, void* stream_) {
     int rc = check_config(cfg);
     if (rc) return rc;
-    if (!hidden_states || !y || !w13_t || !w13s_t || !w2_t || !w2s_t || !workspace)
+    if (!hidden_states || (!y && !o_rows) || !w13_t || !w13s_t || !w2_t || !w2s_t || !workspace)
         return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
     if ((router_logits == nullptr) == (topk_idx == nullptr))
         return fail(MOE_ERR_INVALID_ARG, "moe_forward: pass exactly one of router_logits and topk_idx");
-    if (topk_idx && !topk_weights) return fail(MOE_ERR_INVALID_ARG, "moe_forward: topk_idx needs topk_weights");
-    if (!aligned(hidden_states, 16) || !aligned(y, 16) || !aligned(w13_t, 32) || !aligned(w2_t, 32) ||
+    if (topk_idx && !topk_weights && !o_rows)
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward: topk_idx needs topk_weights");
+    if (!aligned(hidden_states, 16) || !aligned(y ? y : static_cast<void*>(o_rows), 16) || !aligned(w13_t, 32) ||
+        !aligned(w2_t, 32) ||
         !aligned(w13s_t, 16) || !aligned(w2s_t, 16) || !aligned(workspace, 256) ||
         (router_logits && !aligned(router_logits, 4)) || (topk_idx && !aligned(topk_idx, 4)) ||
         (topk_weights && !aligned(topk_weights, 4)) || (w13_bias && !aligned(w13_bias, 16)) ||
@@ -423,10 +429,107 @@ int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, con
                     : (narrow ? moe::launch_gemm_narrow(g2, tm_w2, tm_act, di.sms, s)
                               : moe::launch_gemm(g2, tm_act, tm_w2, di.sms, s)));
     MOE_CUDA_TRY(mark(5));
-    moe::CombineArgs ca{static_cast<const float*>(at(L.o)), static_cast<const int32_t*>(at(L.row_of)), wts,
-                        static_cast<__nv_bfloat16*>(y), T, H, KT, K};
-    MOE_CUDA_TRY(moe::launch_combine(ca, s));
+    if (o_rows) {
+        MOE_CUDA_TRY(moe::launch_rows_f32(static_cast<const float*>(at(L.o)),
+                                          static_cast<const int32_t*>(at(L.row_of)), o_rows, T, H, status, s));
+    } else {
+        moe::CombineArgs ca{static_cast<const float*>(at(L.o)), static_cast<const int32_t*>(at(L.row_of)), wts,
+                            static_cast<__nv_bfloat16*>(y), T, H, KT, K};
+        MOE_CUDA_TRY(moe::launch_combine(ca, s));
+    }
     MOE_CUDA_TRY(mark(6));
+    return ok();
+}
+
+int check_ep(const moe_config_t* cfg, int ranks, const char* who) {
+    if (cfg->shared_experts != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "%s: expert parallelism takes no shared expert", who);
+    if (ranks < 1 || ranks > cfg->num_experts || cfg->num_experts % ranks != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "%s: ranks (%d) must divide num_experts (%d)", who, ranks,
+                    cfg->num_experts);
+    return MOE_OK;
+}
+
+}  // namespace
+
+int moe_forward_profiled(const moe_config_t* cfg, const void* hidden_states, const float* router_logits,
+                         const float* per_expert_scale, const int32_t* topk_idx, const float* topk_weights,
+                         const void* w13_t, const void* w13s_t, const void* w2_t, const void* w2s_t,
+                         const void* w13_bias, const void* w2_bias, void* y, int32_t* expert_counts, void* workspace,
+                         size_t workspace_bytes, moe_profile_t* prof, void* stream_) {
+    if (!y) return fail(MOE_ERR_INVALID_ARG, "moe_forward: NULL pointer");
+    return forward_impl(cfg, hidden_states, router_logits, per_expert_scale, topk_idx, topk_weights, w13_t, w13s_t,
+                        w2_t, w2s_t, w13_bias, w2_bias, y, nullptr, expert_counts, workspace, workspace_bytes, prof,
+                        stream_);
+}
+
+int moe_forward_rows(const moe_config_t* cfg, const void* rows, const int32_t* expert_of_row, const void* w13_t,
+                     const void* w13s_t, const void* w2_t, const void* w2s_t, const void* w13_bias,
+                     const void* w2_bias, float* o_rows, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (cfg->top_k != 1 || cfg->shared_experts != 0)
+        return fail(MOE_ERR_INVALID_ARG, "moe_forward_rows: one slot per row (top_k 1, no shared expert)");
+    if (!rows || !expert_of_row || !o_rows) return fail(MOE_ERR_INVALID_ARG, "moe_forward_rows: NULL pointer");
+    return forward_impl(cfg, rows, nullptr, nullptr, expert_of_row, nullptr, w13_t, w13s_t, w2_t, w2s_t, w13_bias,
+                        w2_bias, nullptr, o_rows, nullptr, workspace, workspace_bytes, nullptr, stream);
+}
+
+int moe_ep_dispatch(const moe_config_t* cfg, int ranks, const void* hidden_states, const int32_t* topk_idx,
+                    int32_t* send_counts, void* send_x, int32_t* send_expert, int32_t* slot_pos, void* workspace,
+                    size_t workspace_bytes, void* stream_) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if ((rc = check_ep(cfg, ranks, "moe_ep_dispatch"))) return rc;
+    if (!hidden_states || !topk_idx || !send_counts || !send_x || !send_expert || !slot_pos || !workspace)
+        return fail(MOE_ERR_INVALID_ARG, "moe_ep_dispatch: NULL pointer");
+    if (!aligned(hidden_states, 16) || !aligned(send_x, 16) || !aligned(topk_idx, 4) || !aligned(send_counts, 4) ||
+        !aligned(send_expert, 4) || !aligned(slot_pos, 4) || !aligned(workspace, 256))
+        return fail(MOE_ERR_INVALID_ARG,
+                    "moe_ep_dispatch: misaligned buffer (rows need 16 bytes, workspace 256, ids 4)");
+    moe_workspace_layout_t L;
+    layout_of(cfg, &L);
+    if (workspace_bytes < L.total)
+        return fail(MOE_ERR_INVALID_ARG, "moe_ep_dispatch: workspace has %zu bytes, needs %zu", workspace_bytes,
+                    L.total);
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    const int T = cfg->num_tokens, K = cfg->top_k, E = cfg->num_experts, A = T * K;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
+    int32_t* status = static_cast<int32_t*>(at(L.status));
+    int32_t* dest = static_cast<int32_t*>(at(L.topk_idx));     // [A], free while topk_idx is the caller's
+    int32_t* row_src = static_cast<int32_t*>(at(L.row_src));
+    cudaStream_t s = static_cast<cudaStream_t>(stream_);
+    MOE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    moe::EpArgs ea{topk_idx, dest, row_src, static_cast<const __nv_bfloat16*>(hidden_states),
+                   static_cast<__nv_bfloat16*>(send_x), send_expert, status, A, K, cfg->hidden, E, E / ranks};
+    MOE_CUDA_TRY(moe::launch_ep_dest(ea, s));
+    // the permutation with the destination ranks as its "experts": counts = send counts,
+    // row_src = send order, row_of = each slot's position in it
+    moe::PermuteArgs pa{dest, static_cast<int32_t*>(at(L.hist)), send_counts, static_cast<int32_t*>(at(L.offsets)),
+                        static_cast<int32_t*>(at(L.tile_start)), row_src, slot_pos, nullptr, status, A, ranks,
+                        moe::permute_chunks(A), moe::permute_chunk_rows(A), T, K, K};
+    if (A <= moe::kSmallRows) MOE_CUDA_TRY(moe::launch_permute_small(pa, false, s));
+    else MOE_CUDA_TRY(moe::launch_permute(pa, s));
+    MOE_CUDA_TRY(moe::launch_ep_gather(ea, s));
+    return ok();
+}
+
+int moe_combine_rows(const moe_config_t* cfg, const float* o_rows, const int32_t* slot_pos,
+                     const float* topk_weights, void* y, void* stream) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (cfg->shared_experts != 0)
+        return fail(MOE_ERR_UNSUPPORTED, "moe_combine_rows: expert parallelism takes no shared expert");
+    if (!o_rows || !slot_pos || !topk_weights || !y) return fail(MOE_ERR_INVALID_ARG, "moe_combine_rows: NULL pointer");
+    if (!aligned(o_rows, 16) || !aligned(y, 16) || !aligned(slot_pos, 4) || !aligned(topk_weights, 4))
+        return fail(MOE_ERR_INVALID_ARG, "moe_combine_rows: misaligned buffer (rows need 16 bytes)");
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    moe::CombineArgs ca{o_rows, slot_pos, topk_weights, static_cast<__nv_bfloat16*>(y), cfg->num_tokens, cfg->hidden,
+                        cfg->top_k, cfg->top_k};
+    MOE_CUDA_TRY(moe::launch_combine(ca, static_cast<cudaStream_t>(stream)));
     return ok();
 }
 

@@ -121,6 +121,10 @@ def _load():
             lib.orc_scaled_gemv.argtypes = [ctypes.c_int] * 3 + [P] * 5
             lib.orc_forward.restype = ctypes.c_int
             lib.orc_forward.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 11 + [P, ctypes.c_int, P, P, P]
+            lib.orc_expert_rows.restype = ctypes.c_int
+            lib.orc_expert_rows.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int] + [P] * 9
+            lib.orc_combine_rows.restype = ctypes.c_int
+            lib.orc_combine_rows.argtypes = [ctypes.c_int] * 3 + [P] * 4
             lib.orc_forward_permuted.restype = ctypes.c_int
             lib.orc_forward_permuted.argtypes = [ctypes.POINTER(_Cfg)] + [P] * 10
             lib.orc_quantize_tokens.restype = None
@@ -289,6 +293,38 @@ def forward(cfg: Config, x_bf16, w13, w13s, w2, w2s, logits=None, per_expert_sca
     if rc:
         raise ValueError(f"oracle forward: invalid configuration ({rc})")
     return (y, act_q, act_s) if want_act else y
+
+
+def expert_rows(cfg: Config, x_bf16, expert_of_row, w13, w13s, w2, w2s, b13=None, b2=None) -> np.ndarray:
+    """Expert parallelism, the owning rank's side: each row x_n (bf16 bits) quantized as the layer
+    does, then through expert e_n's MLP (local numbering; cfg.num_experts = that rank's experts).
+    Returns the fp64 outputs [N, H] (before the routing weight)."""
+    x = _arr(x_bf16, np.uint16)
+    e = _arr(expert_of_row, np.int32)
+    N = int(e.size)
+    sd = cfg.scale_dtype
+    o = np.zeros((N, cfg.hidden), np.float64)
+    rc = _load().orc_expert_rows(ctypes.byref(cfg.c()), N, _p(x), _p(e), _p(_arr(w13, np.uint8)), _p(_arr(w13s, sd)),
+                                 _p(_arr(w2, np.uint8)), _p(_arr(w2s, sd)), _p(_arr(b13, np.uint16)),
+                                 _p(_arr(b2, np.uint16)), _p(o))
+    if rc:
+        raise ValueError(f"oracle expert_rows: expert id out of range ({rc})")
+    return o
+
+
+def combine_rows(o_rows, slot_pos, topk_weights) -> np.ndarray:
+    """Expert parallelism, the home rank's side: y_t = bf16(sum_j w_tj * o[pos_tj]) in slot order
+    (fp64 sum).  o_rows fp64 [T*k, H], slot_pos int32 [T, k], topk_weights fp32 [T, k]."""
+    o = _arr(o_rows, np.float64)
+    pos = _arr(slot_pos, np.int32)
+    w = _arr(topk_weights, np.float32)
+    T, K = pos.shape
+    H = o.shape[1]
+    y = np.zeros((T, H), np.uint16)
+    rc = _load().orc_combine_rows(T, K, H, _p(o), _p(pos), _p(w), _p(y))
+    if rc:
+        raise ValueError(f"oracle combine_rows: position out of range ({rc})")
+    return y
 
 
 def forward_permuted(cfg: Config, x_bf16, w13, w13s, w2, w2s, logits, per_expert_scale=None,

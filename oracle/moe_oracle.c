@@ -575,6 +575,60 @@ int orc_forward(const orc_cfg *c, const uint16_t *x, const float *logits,
 }
 
 /* ------------------------------------------------------------------------------------------
+ * Expert parallelism, the two sides of the exchange ([MindIE] execution flow: dispatch, mlp,
+ * combine; the dynamic dispatcher's all-to-all).  A rank that owns some experts receives token
+ * rows, each tagged with one of its experts, and returns each row's expert output; the token's
+ * home rank then forms the weighted sum.
+ *
+ * orc_expert_rows: for each row n, quantize x_n as the layer does and run expert e_n's MLP:
+ *   o[n] = expert_mlp(quantize(x_n), e_n)                    (fp64, H values)
+ * c describes the owning rank: num_experts = its experts, weights indexed by local id.
+ * Returns ORC_EINVAL for an expert id outside [0, num_experts).
+ * ---------------------------------------------------------------------------------------- */
+int orc_expert_rows(const orc_cfg *c, int N, const uint16_t *x, const int32_t *expert_of_row,
+                    const uint8_t *w13, const void *w13s, const uint8_t *w2, const void *w2s,
+                    const uint16_t *b13, const uint16_t *b2, double *o)
+{
+    const int H = c->hidden, g = c->recipe == 0 ? 128 : 32;
+    const size_t sb = scale_bytes(c->recipe);
+    orc_weights W = {w13, w13s, w2, w2s, b13, b2};
+    int bad = 0;
+    for (int n = 0; n < N; n++)
+        if (expert_of_row[n] < 0 || expert_of_row[n] >= c->num_experts) bad = 1;
+    if (bad) return ORC_EINVAL;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < N; n++) {
+        float *xf = (float *)malloc(sizeof(float) * (size_t)H);
+        uint8_t *xq = (uint8_t *)malloc((size_t)H);
+        void *xs = malloc(sb * (size_t)(H / g));
+        for (int h = 0; h < H; h++) xf[h] = bf16_to_f32(x[(size_t)n * H + h]);
+        orc_quant_row(xf, H, c->recipe, xq, xs);
+        expert_mlp_row(c, &W, expert_of_row[n], xq, xs, o + (size_t)n * H, NULL, NULL);
+        free(xf); free(xq); free(xs);
+    }
+    return ORC_OK;
+}
+
+/* orc_combine_rows: on the home rank, y_t = bf16_rn( sum_j w_tj * o[pos_tj] ), the sum in fp64
+ * in slot order j = 0..K-1, as in orc_forward.  pos indexes the A = T*K returned rows. */
+int orc_combine_rows(int T, int K, int H, const double *o, const int32_t *pos, const float *w,
+                     uint16_t *y)
+{
+    const int A = T * K;
+    for (int i = 0; i < A; i++)
+        if (pos[i] < 0 || pos[i] >= A) return ORC_EINVAL;
+    for (int t = 0; t < T; t++)
+        for (int h = 0; h < H; h++) {
+            double acc = 0.0;
+            for (int j = 0; j < K; j++)
+                acc += (double)w[(size_t)t * K + j] * o[(size_t)pos[(size_t)t * K + j] * H + h];
+            y[(size_t)t * H + h] = orc_bf16_from_double(acc);
+        }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------------------------
  * The same forward through the permuted formulation: route all tokens, permute rows into
  * expert-contiguous order, run each expert over its rows, then combine back in token order.
  * Used to check that the per-token loop and the dispatch/combine plumbing agree bit for bit.
