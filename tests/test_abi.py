@@ -146,3 +146,30 @@ def test_gate_entry_points_validate_before_any_cuda_call():
     bad = moe.Config(num_tokens=0, hidden=384, inter=128, num_experts=24, top_k=3).c()
     n = ctypes.c_size_t(0)
     assert lib.moe_gate_weights_size(ctypes.byref(bad), ctypes.byref(n)) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_expert_parallel_entry_points_validate_before_any_cuda_call():
+    """Ranks must divide the expert count, no shared expert, one slot per row on the expert side,
+    no NULL buffers: each rejected with a message and nothing launched."""
+    lib = moe.lib()
+    buf = ctypes.create_string_buffer(4096)
+    al = (ctypes.addressof(buf) + 255) & ~255
+    c = cfg(num_experts=8, top_k=2).c()
+    rc = lib.moe_ep_dispatch(ctypes.byref(c), 3, al, al, al, al, al, al, al, 1 << 20, None)
+    assert rc == moe.MOE_ERR_UNSUPPORTED and b"divide" in lib.moe_last_error()
+    rc = lib.moe_ep_dispatch(ctypes.byref(c), 2, None, al, al, al, al, al, al, 1 << 20, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"NULL" in lib.moe_last_error()
+    rc = lib.moe_ep_dispatch(ctypes.byref(c), 2, al, al, al, al, al, al, al, 16, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"workspace" in lib.moe_last_error()
+    sh = cfg(num_experts=8, top_k=2, shared_experts=1).c()
+    rc = lib.moe_ep_dispatch(ctypes.byref(sh), 2, al, al, al, al, al, al, al, 1 << 20, None)
+    assert rc == moe.MOE_ERR_UNSUPPORTED and b"shared" in lib.moe_last_error()
+    rc = lib.moe_forward_rows(ctypes.byref(c), al, al, al, al, al, al, None, None, al, al, 1 << 20, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"one slot per row" in lib.moe_last_error()
+    one = cfg(num_experts=4, top_k=1).c()
+    rc = lib.moe_forward_rows(ctypes.byref(one), al, None, al, al, al, al, None, None, al, al, 1 << 20, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"NULL" in lib.moe_last_error()
+    rc = lib.moe_combine_rows(ctypes.byref(c), al, None, al, al, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"NULL" in lib.moe_last_error()
+    rc = lib.moe_combine_rows(ctypes.byref(c), al | 4, al, al, al, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"misaligned" in lib.moe_last_error()
