@@ -1,6 +1,8 @@
 /*
- * moefp8.h -- C ABI of libmoefp8.so: the forward of one fused routed-expert FP8 MoE layer on a
- * single NVIDIA B200 (sm_100a).
+ * moefp8.h -- C ABI of libmoefp8.so: the forward of one fused routed-expert FP8 MoE layer on
+ * NVIDIA B200 (sm_100a): the whole layer on one GPU (moe_forward), the gate in front of its
+ * router (moe_gate), and the device steps of expert parallelism over the GPUs of a node
+ * (moe_ep_dispatch, moe_forward_rows, moe_combine_rows), around an all-to-all the caller runs.
  *
  * The layer (sources are web pages, cited by title and section):
  *   "MindIE-SD Fused MoE" -- function signature and parameter table (hidden_states,
