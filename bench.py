@@ -269,6 +269,66 @@ def gate_only(args, shape, local):
     print(json.dumps(line))
 
 
+class LocalExchange:
+    """The all-to-all of a single rank: every row stays home (what ep_step sees at N = 1)."""
+
+    @staticmethod
+    def all_to_all_single(out, inp, out_splits=None, in_splits=None, group=None):
+        out.copy_(inp)
+
+
+def ep_bench(args, shape, world, rank, local, dist):
+    """Expert parallelism (mixture_experts_fp8_b200.ep): every rank owns E/N experts and routes its
+    own batch of the problem's size; one step = route, dispatch, all-to-all, the expert side,
+    the reverse all-to-all, combine.  Times K steps with CUDA events, max over ranks."""
+    import mixture_experts_fp8_b200 as moe
+    from mixture_experts_fp8_b200 import ep
+
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    from dataclasses import replace
+    shape = replace(shape, seed=shape.seed + 1000 * rank)           # each rank its own tokens
+    prob = synth.make_problem(shape, device=dev)
+    e_loc = shape.num_experts // world
+    es = slice(rank * e_loc, (rank + 1) * e_loc)
+    cfg = moe.Config(**shape.cfg())
+    cfg_w = ep.rows_config(cfg, world, 1)
+    w_local = moe.transform_weights(cfg_w, prob.w13[es].contiguous(), prob.w13_scale[es].contiguous(),
+                                    prob.w2[es].contiguous(), prob.w2_scale[es].contiguous())
+    b13 = None if prob.w13_bias is None else prob.w13_bias[es].contiguous()
+    b2 = None if prob.w2_bias is None else prob.w2_bias[es].contiguous()
+    ws = moe.new_workspace(cfg, dev)
+    exch = dist if dist is not None else LocalExchange()
+
+    def step():
+        return ep.ep_step(cfg, world, prob.x, prob.logits, w_local, exch, per_expert_scale=prob.per_expert_scale,
+                          w13_bias_local=b13, w2_bias_local=b2, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        y, stats = step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = reduce_max(a.elapsed_time(b), dist, dev)
+    if rank == 0:
+        line = {"metric": "MoE-layer tokens/s, expert parallel", "value": job_tokens_per_s(world, shape.num_tokens,
+                                                                                      args.steps, ms),
+                "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "e4m3", "data": "synthetic",
+                "config": {"workload": describe(shape) + f"; expert parallel over {world} rank(s), "
+                                                         f"{e_loc} experts each",
+                           "exchange": "torch.distributed all_to_all_single" if dist else "none (one rank)"},
+                "ep": {"rows_sent_by_rank0": stats["sent"], "rows_received_by_rank0": stats["received"]}}
+        print(json.dumps(line))
+
+
 def reference_arm(args, shape, rank):
     if rank != 0:
         return
@@ -312,6 +372,8 @@ def main():
     ap.add_argument("--gate", action="store_true",
                     help="start each step from the gate (RMSNorm + router matmul + top-k, moe_gate) on "
                          "the bf16 hidden states instead of from precomputed router logits")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism: every rank owns num_experts/N experts and routes its own batch")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every kernel from the host instead of replaying a captured CUDA graph")
     ap.add_argument("--gate-only", action="store_true",
@@ -338,6 +400,20 @@ def main():
     if args.gate_only:
         if rank == 0:
             gate_only(args, shape, local)
+        return
+    if args.ep:
+        dist = None
+        if world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        try:
+            ep_bench(args, shape, world, rank, local, dist)
+        finally:
+            if dist:
+                dist.destroy_process_group()
         return
 
     import mixture_experts_fp8_b200 as moe
