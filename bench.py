@@ -287,8 +287,8 @@ def ep_bench(args, shape, world, rank, local, dist):
     torch.cuda.set_device(local)
     dev = f"cuda:{local}"
     from dataclasses import replace
-    shape = replace(shape, seed=shape.seed + 1000 * rank)           # each rank its own tokens
-    prob = synth.make_problem(shape, device=dev)
+    prob = synth.make_problem(shape, device=dev)                    # the same layer on every rank
+    x, logits, _ = synth.make_activations(replace(shape, seed=shape.seed + 1000 * rank), device=dev)  # its tokens
     e_loc = shape.num_experts // world
     es = slice(rank * e_loc, (rank + 1) * e_loc)
     cfg = moe.Config(**shape.cfg())
@@ -301,7 +301,7 @@ def ep_bench(args, shape, world, rank, local, dist):
     exch = dist if dist is not None else LocalExchange()
 
     def step():
-        return ep.ep_step(cfg, world, prob.x, prob.logits, w_local, exch, per_expert_scale=prob.per_expert_scale,
+        return ep.ep_step(cfg, world, x, logits, w_local, exch, per_expert_scale=prob.per_expert_scale,
                           w13_bias_local=b13, w2_bias_local=b2, workspace=ws)
 
     for _ in range(args.warmup):
