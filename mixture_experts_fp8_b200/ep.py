@@ -90,7 +90,8 @@ def ep_step(cfg, ranks: int, x, router_logits, weights_local, dist, group=None, 
     sc = send_counts.to(torch.int64)
     rc = torch.empty_like(sc)
     dist.all_to_all_single(rc, sc, group=group)
-    send_splits, recv_splits = [int(v) for v in sc.tolist()], [int(v) for v in rc.tolist()]
+    both = torch.stack([sc, rc]).tolist()          # one read-back of both split lists
+    send_splits, recv_splits = [int(v) for v in both[0]], [int(v) for v in both[1]]
     recv_x = all_to_all_rows(dist, group, send_x[:sum(send_splits)], send_splits, recv_splits)
     recv_e = all_to_all_rows(dist, group, send_expert[:sum(send_splits)], send_splits, recv_splits)
 
