@@ -165,3 +165,23 @@ def test_two_rank_exchange_matches_the_single_process_forward(name, tmp_path):
     assert all(stats[a]["sent"][b] == stats[b]["received"][a] for a in range(2) for b in range(2))
     if name == "one_sided":
         assert sum(stats[1]["received"]) == 0
+
+
+def test_one_rank_with_the_benchmark_local_exchange():
+    """World size 1 (what bench.py --ep runs without torchrun): every row stays home, through
+    bench.LocalExchange; the result is the single-process forward."""
+    import bench
+
+    import mixture_experts_fp8_b200 as moe
+    from mixture_experts_fp8_b200 import ep
+
+    shape, prob = _problem("groups")
+    ni = prob.numpy_inputs()
+    cfg = moe.Config(**shape.cfg())
+    y, stats = ep.ep_step(cfg, 1, prob.x, prob.logits, (ni["w13"], ni["w13s"], ni["w2"], ni["w2s"]),
+                          bench.LocalExchange(), ops=OracleOps(), per_expert_scale=prob.per_expert_scale,
+                          w13_bias_local=ni["b13"], w2_bias_local=ni["b2"])
+    ref = oracle.forward(oracle.Config(**shape.cfg()), ni["x"], ni["w13"], ni["w13s"], ni["w2"], ni["w2s"],
+                         logits=ni["logits"], per_expert_scale=ni["per_expert_scale"], b13=ni["b13"], b2=ni["b2"])
+    assert np.array_equal(y.numpy(), ref)
+    assert stats["sent"] == stats["received"] == [shape.num_tokens * shape.top_k]
