@@ -113,6 +113,10 @@ def _load():
             lib.orc_check_cfg.argtypes = [ctypes.POINTER(_Cfg)]
             lib.orc_route.restype = ctypes.c_int
             lib.orc_route.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P, P]
+            lib.orc_group_scores.restype = ctypes.c_int
+            lib.orc_group_scores.argtypes = [ctypes.POINTER(_Cfg), P, P]
+            lib.orc_route_weights.restype = ctypes.c_int
+            lib.orc_route_weights.argtypes = [ctypes.POINTER(_Cfg), P, P, P, P]
             lib.orc_gate_logits.restype = None
             lib.orc_gate_logits.argtypes = [ctypes.c_int] * 3 + [P] * 3 + [ctypes.c_float, P]
             lib.orc_permute.restype = None
@@ -227,6 +231,30 @@ def route(cfg: Config, logits: np.ndarray, per_expert_scale=None):
     if rc:
         raise ValueError(f"oracle route: invalid configuration ({rc})")
     return idx, w, tie
+
+
+def group_scores(cfg: Config, logits: np.ndarray) -> np.ndarray:
+    """-> fp32 group scores [T, group_count], the values the group choice is taken on."""
+    logits = _arr(logits, np.float32)
+    g = np.zeros((cfg.num_tokens, cfg.group_count), np.float32)
+    c = cfg.c()
+    rc = _load().orc_group_scores(ctypes.byref(c), _p(logits), _p(g))
+    if rc:
+        raise ValueError(f"oracle group_scores: invalid configuration ({rc})")
+    return g
+
+
+def route_weights(cfg: Config, logits: np.ndarray, topk_idx: np.ndarray, per_expert_scale=None) -> np.ndarray:
+    """-> fp32 [T, k]: the routing weights of the given expert ids under cfg's weight rule."""
+    logits = _arr(logits, np.float32)
+    idx = _arr(topk_idx, np.int32)
+    pes = _arr(per_expert_scale, np.float32)
+    w = np.zeros((cfg.num_tokens, cfg.top_k), np.float32)
+    c = cfg.c()
+    rc = _load().orc_route_weights(ctypes.byref(c), _p(logits), _p(pes), _p(idx), _p(w))
+    if rc:
+        raise ValueError(f"oracle route_weights: invalid configuration or ids ({rc})")
+    return w
 
 
 def permute(topk_idx: np.ndarray, num_experts: int):

@@ -271,6 +271,69 @@ int orc_check_cfg(const orc_cfg *c)
     return ORC_OK;
 }
 
+/* fp32 scores of one token's experts (used only for the group scores): sigmoid, or softmax
+ * over all E. */
+static void token_scores(const orc_cfg *c, const float *l, float *score)
+{
+    const int E = c->num_experts;
+    if (c->routing == 1) {
+        for (int e = 0; e < E; e++) score[e] = 1.0f / (1.0f + expf(-l[e]));
+    } else {
+        float m = l[0], z = 0.0f;
+        for (int e = 1; e < E; e++) m = fmaxf(m, l[e]);
+        for (int e = 0; e < E; e++) z += expf(l[e] - m);
+        for (int e = 0; e < E; e++) score[e] = expf(l[e] - m) / z;
+    }
+}
+
+/* fp32 group scores of one token from its expert scores: the max of the group's scores
+ * (mode 0) or the sum of its two largest (mode 1). */
+static void group_scores(const orc_cfg *c, const float *score, float *gscore)
+{
+    const int G = c->group_count, gs = c->num_experts / G;
+    for (int g = 0; g < G; g++) {
+        const float *s = score + g * gs;
+        if (c->group_select_mode == 0) {
+            float mx = s[0];
+            for (int i = 1; i < gs; i++) mx = fmaxf(mx, s[i]);
+            gscore[g] = mx;
+        } else {
+            int i1 = 0, i2 = -1;
+            for (int i = 1; i < gs; i++) if (s[i] > s[i1]) i1 = i;
+            for (int i = 0; i < gs; i++)
+                if (i != i1 && (i2 < 0 || s[i] > s[i2])) i2 = i;
+            gscore[g] = s[i1] + s[i2];
+        }
+    }
+}
+
+/* Weights of the selected experts ids[k] of one token, in fp64, rounded once to fp32. */
+static void route_weights(const orc_cfg *c, const float *l, const float *per_expert_scale,
+                          const int32_t *ids, float *w)
+{
+    const int E = c->num_experts, K = c->top_k;
+    double wsum = 0.0, wd[256];
+    if (c->routing == 1) {
+        for (int j = 0; j < K; j++) wd[j] = 1.0 / (1.0 + exp(-(double)l[ids[j]]));
+        for (int j = 0; j < K; j++) wsum += wd[j];
+        for (int j = 0; j < K; j++) wd[j] /= wsum;
+    } else {
+        double m = l[0], z = 0.0;
+        for (int e = 1; e < E; e++) m = fmax(m, (double)l[e]);
+        for (int e = 0; e < E; e++) z += exp((double)l[e] - m);
+        for (int j = 0; j < K; j++) wd[j] = exp((double)l[ids[j]] - m) / z;
+        if (c->renormalize) {
+            for (int j = 0; j < K; j++) wsum += wd[j];
+            for (int j = 0; j < K; j++) wd[j] /= wsum;
+        }
+    }
+    for (int j = 0; j < K; j++) {
+        if (per_expert_scale) wd[j] *= (double)per_expert_scale[ids[j]];
+        wd[j] *= (double)c->routed_scaling_factor;
+        w[j] = (float)wd[j];
+    }
+}
+
 /* Route one token: logits l[E] -> ids[k], weights[k]; returns 1 if the group choice was a
  * near tie, else 0. */
 static int route_token(const orc_cfg *c, const float *l, const float *per_expert_scale,
@@ -280,38 +343,15 @@ static int route_token(const orc_cfg *c, const float *l, const float *per_expert
     float score[256];
     unsigned char eligible[256], taken[256];
     int near_tie = 0;
-    double wsum = 0.0, wd[256];
 
-    /* fp32 scores, used only for the group scores. */
-    if (c->routing == 1) {
-        for (int e = 0; e < E; e++) score[e] = 1.0f / (1.0f + expf(-l[e]));
-    } else {
-        float m = l[0], z = 0.0f;
-        for (int e = 1; e < E; e++) m = fmaxf(m, l[e]);
-        for (int e = 0; e < E; e++) z += expf(l[e] - m);
-        for (int e = 0; e < E; e++) score[e] = expf(l[e] - m) / z;
-    }
-
+    token_scores(c, l, score);
     for (int e = 0; e < E; e++) eligible[e] = 1;
     if (G > 1) {
         float gscore[256];
         unsigned char gtaken[256];
         int order[256];
-        for (int g = 0; g < G; g++) {
-            const float *s = score + g * gs;
-            if (c->group_select_mode == 0) {
-                float mx = s[0];
-                for (int i = 1; i < gs; i++) mx = fmaxf(mx, s[i]);
-                gscore[g] = mx;
-            } else {
-                int i1 = 0, i2 = -1;
-                for (int i = 1; i < gs; i++) if (s[i] > s[i1]) i1 = i;
-                for (int i = 0; i < gs; i++)
-                    if (i != i1 && (i2 < 0 || s[i] > s[i2])) i2 = i;
-                gscore[g] = s[i1] + s[i2];
-            }
-            gtaken[g] = 0;
-        }
+        group_scores(c, score, gscore);
+        for (int g = 0; g < G; g++) gtaken[g] = 0;
         for (int r = 0; r < G; r++) {                 /* full order of groups */
             int best = -1;
             for (int g = 0; g < G; g++)
@@ -336,28 +376,41 @@ static int route_token(const orc_cfg *c, const float *l, const float *per_expert
         ids[j] = best;
         taken[best] = 1;
     }
-
-    /* weights, in fp64 */
-    if (c->routing == 1) {
-        for (int j = 0; j < K; j++) wd[j] = 1.0 / (1.0 + exp(-(double)l[ids[j]]));
-        for (int j = 0; j < K; j++) wsum += wd[j];
-        for (int j = 0; j < K; j++) wd[j] /= wsum;
-    } else {
-        double m = l[0], z = 0.0;
-        for (int e = 1; e < E; e++) m = fmax(m, (double)l[e]);
-        for (int e = 0; e < E; e++) z += exp((double)l[e] - m);
-        for (int j = 0; j < K; j++) wd[j] = exp((double)l[ids[j]] - m) / z;
-        if (c->renormalize) {
-            for (int j = 0; j < K; j++) wsum += wd[j];
-            for (int j = 0; j < K; j++) wd[j] /= wsum;
-        }
-    }
-    for (int j = 0; j < K; j++) {
-        if (per_expert_scale) wd[j] *= (double)per_expert_scale[ids[j]];
-        wd[j] *= (double)c->routed_scaling_factor;
-        w[j] = (float)wd[j];
-    }
+    route_weights(c, l, per_expert_scale, ids, w);
     return near_tie;
+}
+
+/* The fp32 group scores of every token, [T, group_count] (the values the near-tie flag and
+ * the group choice above are taken on); for checking another implementation's group choice. */
+int orc_group_scores(const orc_cfg *c, const float *logits, float *gscores)
+{
+    int rc = orc_check_cfg(c);
+    if (rc) return rc;
+    const int E = c->num_experts, G = c->group_count;
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < c->num_tokens; t++) {
+        float score[256];
+        token_scores(c, logits + (size_t)t * E, score);
+        group_scores(c, score, gscores + (size_t)t * G);
+    }
+    return ORC_OK;
+}
+
+/* Routing weights of caller-chosen experts topk_idx [T, k] (each id in [0, E)): the same
+ * weight rule as orc_route, for checking the weights that go with another implementation's
+ * valid selection. */
+int orc_route_weights(const orc_cfg *c, const float *logits, const float *per_expert_scale,
+                      const int32_t *topk_idx, float *topk_w)
+{
+    int rc = orc_check_cfg(c);
+    if (rc) return rc;
+    for (size_t i = 0; i < (size_t)c->num_tokens * c->top_k; i++)
+        if (topk_idx[i] < 0 || topk_idx[i] >= c->num_experts) return ORC_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < c->num_tokens; t++)
+        route_weights(c, logits + (size_t)t * c->num_experts, per_expert_scale,
+                      topk_idx + (size_t)t * c->top_k, topk_w + (size_t)t * c->top_k);
+    return ORC_OK;
 }
 
 int orc_route(const orc_cfg *c, const float *logits, const float *per_expert_scale,

@@ -275,3 +275,21 @@ def random_shape(seed: int, **over) -> Shape:
               routed_scaling_factor=float(rng.choice([1.0, 2.5])),
               per_expert_scale=bool(rng.integers(0, 2)), biases=bool(rng.integers(0, 2)))
     return replace(s, **over)
+
+
+def random_grouped_shape(seed: int, **over) -> Shape:
+    """A small ragged problem with grouped routing: the experts form group_count groups, the
+    k_group best (max or top-2-sum group score) are kept, top_k is chosen inside them."""
+    rng = np.random.default_rng(2000 + seed)
+    E = int(rng.choice([8, 16, 32, 64]))
+    G = int(rng.choice([g for g in (2, 4, 8) if E % g == 0 and E // g >= 2]))
+    kg = int(rng.integers(1, G + 1))
+    k = int(rng.integers(1, min(8, kg * (E // G)) + 1))
+    s = Shape(f"grp{seed}", num_tokens=int(rng.choice([5, 64, 129, 300])),
+              hidden=int(rng.choice([128, 256, 384])), inter=int(rng.choice([128, 256])),
+              num_experts=E, top_k=k, routing=int(rng.integers(0, 2)),
+              renormalize=int(rng.integers(0, 2)), group_count=G, k_group=kg,
+              group_select_mode=int(rng.integers(0, 2)), recipe=int(rng.integers(0, 3)),
+              seed=20_000 + seed, routed_scaling_factor=float(rng.choice([1.0, 2.5])),
+              logit_bias_std=float(rng.choice([0.0, 0.1])), biases=bool(rng.integers(0, 2)))
+    return replace(s, **over)

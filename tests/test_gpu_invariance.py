@@ -18,9 +18,11 @@ from _helpers import GpuProblem, bits, lib_cfg
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "skewed"])
+@pytest.mark.parametrize("name", ["tiny", "decode", "skewed", "prefill", "large"])
 def test_batch_invariance(name):
-    prob = synth.make_problem(name)
+    """Full-size prefill and large run the wide kernels on the full batch and on the half batch,
+    the narrow (swap-AB) kernels on the single tokens."""
+    prob = synth.make_problem(name, device="cuda" if name in ("prefill", "large") else "cpu")
     gp = GpuProblem(prob)
     y_full = bits(gp.forward())
     T = prob.shape.num_tokens

@@ -24,8 +24,8 @@ from _helpers import (GpuProblem, assert_y_close, bits, check_routing, oracle_cf
 pytestmark = pytest.mark.gpu
 
 FULL = ["tiny", "decode", "prefill", "skewed", "large", "decode_w4a8", "prefill_w4a8"]
-SAMPLE_TOKENS = {"tiny": None, "decode": None, "skewed": 384, "prefill": 48, "large": 96,
-                 "decode_w4a8": None, "prefill_w4a8": 48}
+SAMPLE_TOKENS = {"tiny": None, "decode": None, "skewed": 384, "prefill": 128, "large": 256,
+                 "decode_w4a8": None, "prefill_w4a8": 128}
 ON_GPU = ("prefill", "large", "prefill_w4a8")     # inputs drawn on the device (their size)
 
 
@@ -95,7 +95,7 @@ def test_permutation_and_quantization(problems, name):
         assert np.array_equal(xs[rows], s_ref), f"scales differ (slot {j})"
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "skewed", "large"])
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed", "large", "prefill_w4a8"])
 def test_gate_up_swiglu_codes(problems, name):
     """The gate+up GEMM's requantized SwiGLU products (E4M3 codes and scales) against the
     oracle's, per routed row: codes may differ by one step where the fp32 and fp64 sums straddle a
@@ -142,9 +142,10 @@ def test_forward_output(problems, name):
     idx_g = idx_g.reshape(shape.num_tokens, shape.top_k)
     w_g = w_g.reshape(shape.num_tokens, shape.top_k)
     tok = _sample(shape.num_tokens, SAMPLE_TOKENS[name], 11)
-    # Near-tie tokens: the oracle follows the GPU's (valid) choice of experts.
-    _, _, tie = oracle.route(oracle_cfg(shape), ni["logits"], ni["per_expert_scale"])
-    if tie.any():
+    # Near-tie tokens: the GPU's choice of experts must be valid (check_routing), and the oracle
+    # then follows it.
+    nd, nt = check_routing(shape, ni, idx_g, w_g)
+    if nd:
         r = oracle_y(gp.prob, ni, tokens=tok, topk_idx=idx_g, topk_w=w_g)
     else:
         r = oracle_y(gp.prob, ni, tokens=tok)
@@ -154,15 +155,23 @@ def test_forward_output(problems, name):
     print(f"{name}: {m}")
 
 
-@pytest.mark.parametrize("seed,recipe", [(s, None) for s in range(8)] + [(s, 2) for s in range(8, 12)])
+@pytest.mark.parametrize("seed,recipe", [(s, None) for s in range(8)] + [(s, 2) for s in range(8, 12)] +
+                         [(s, "grouped") for s in range(12, 18)])
 def test_forward_random_small(seed, recipe):
-    shape = synth.random_shape(seed) if recipe is None else synth.random_shape(seed, recipe=recipe)
+    if recipe == "grouped":
+        shape = synth.random_grouped_shape(seed)
+    else:
+        shape = synth.random_shape(seed) if recipe is None else synth.random_shape(seed, recipe=recipe)
     prob = synth.make_problem(shape)
     gp = GpuProblem(prob)
     ni = oracle_inputs(prob)
     y = gp.forward()
     assert gp.status() == 0
-    r = oracle_y(prob, ni)
+    T, K = shape.num_tokens, shape.top_k
+    idx_g = gp.ws_region("topk_idx", torch.int32, T * K).cpu().numpy().reshape(T, K)
+    w_g = gp.ws_region("topk_weights", torch.float32, T * K).cpu().numpy().reshape(T, K)
+    nd, _ = check_routing(shape, ni, idx_g, w_g)
+    r = oracle_y(prob, ni, topk_idx=idx_g, topk_w=w_g) if nd else oracle_y(prob, ni)
     assert_y_close(bits(y), r, shape.name)
 
 
