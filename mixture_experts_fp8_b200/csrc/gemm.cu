@@ -302,6 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive_lane0(tempty0 + 8 * buf, lane);
                 fma_chunk16(acc2, vb, ws + 4 * kHalf + 64, 48, sa2);
+                // the scales were read through the generic proxy; the producer's next bulk copy
+                // into this stage is an async-proxy write: order the reads before it
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 mbar_arrive_lane0(empty0 + 8 * s, lane);   // done with the stage's scales
                 if (++s == kStages) {
                     s = 0;

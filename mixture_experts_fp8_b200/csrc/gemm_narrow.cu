@@ -272,6 +272,9 @@ __global__ void __launch_bounds__(kNThreads, 1)
                     if (lane == 0) mbar_arrive(&tempty[b]);
                 }
                 if (!ok) break;
+                // The stage's scales were read through the generic proxy; the producer's next bulk
+                // copy into this stage is an async-proxy write.  Order the reads before it.
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);
             }

@@ -5,9 +5,10 @@
 // slot k the shared expert when there is one); inside an expert, rows keep ascending a (hence
 // ascending token).  The shared expert (index E) holds every token, so its count (T) and its
 // rows (token order) are known without counting; it is appended after the routed experts.
-// Three launches, no global atomics, so the result is the same bits on every run:
+// Three launches, no atomics at all, so the result is the same bits on every run:
 //   1. k_hist     per-chunk expert histograms (a chunk is a multiple of kPermuteChunk routed
-//                 rows, sized so that there are at most kMaxPermuteChunks chunks)
+//                 rows, sized so that there are at most kMaxPermuteChunks chunks), counted per
+//                 warp with a warp match and a population count
 //   2. k_scan     per-expert exclusive bases across chunks, counts, offsets = exclusive scan,
 //                 and the first 128-row GEMM tile of every expert
 //   3. k_scatter  one warp per chunk walks its rows in order; rows with the same expert inside
@@ -18,22 +19,38 @@
 
 namespace moe {
 
+// Count 32 ids of one warp into the warp's own histogram without atomics: lanes holding the same
+// expert find each other with a warp match, and the lowest of them adds the group's size.  Ids
+// outside [0, E) (the shared slot's marker included) are not counted; other ids outside [0, E)
+// set MOE_ERR_BOUNDS.
+__device__ __forceinline__ void warp_count(int* hist_w, int e, bool valid, const PermuteArgs& a) {
+    const int lane = threadIdx.x & 31;
+    if (valid && e != kSharedSlot && (e < 0 || e >= a.E)) set_status(a.status, MOE_ERR_BOUNDS);
+    const int key = valid && e >= 0 && e < a.E ? e : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, key);
+    if (key >= 0 && lane == __ffs(peers) - 1) hist_w[key] += __popc(peers);
+    __syncwarp();
+}
+
 __global__ void __launch_bounds__(256) k_hist(PermuteArgs a) {
-    __shared__ int cnt[MOE_MAX_EXPERTS];
+    __shared__ int cnt[8][MOE_MAX_EXPERTS];            // one histogram per warp
     pdl_wait_then_release();
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x) cnt[e] = 0;
-    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = lane; e < a.E; e += 32) cnt[warp][e] = 0;
+    __syncwarp();
     const int begin = blockIdx.x * a.chunk;
     const int end = min(a.A, begin + a.chunk);
-    for (int r = begin + threadIdx.x; r < end; r += blockDim.x) {
-        const int e = slot_expert(a, r);
-        if (e == kSharedSlot) continue;
-        if (e >= 0 && e < a.E) atomicAdd(&cnt[e], 1);
-        else set_status(a.status, MOE_ERR_BOUNDS);
+    for (int r0 = begin + 32 * warp; r0 < end; r0 += 256) {
+        const int r = r0 + lane;
+        warp_count(cnt[warp], r < end ? slot_expert(a, r) : -1, r < end, a);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < a.E; e += blockDim.x)
-        a.hist[static_cast<size_t>(blockIdx.x) * a.E + e] = cnt[e];
+    for (int e = threadIdx.x; e < a.E; e += blockDim.x) {
+        int sum = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) sum += cnt[w][e];
+        a.hist[static_cast<size_t>(blockIdx.x) * a.E + e] = sum;
+    }
 }
 
 // Exclusive scan of v over the 256 threads of the block (v of threads >= n treated as 0).
@@ -172,11 +189,9 @@ __global__ void __launch_bounds__(kSmallWarps * 32) k_permute_small(PermuteArgs 
     __syncthreads();
     const int C = ((A + kSmallWarps - 1) / kSmallWarps + 31) / 32 * 32;
     const int begin = warp * C, end = min(A, begin + C);
-    for (int r = begin + lane; r < end; r += 32) {
-        const int e = ids[r];
-        if (e == kSharedSlot) continue;
-        if (e >= 0 && e < E) atomicAdd(&hist[warp * E + e], 1);
-        else set_status(pa.status, MOE_ERR_BOUNDS);
+    for (int r0 = begin; r0 < end; r0 += 32) {         // each warp counts its own chunk
+        const int r = r0 + lane;
+        warp_count(hist + warp * E, r < end ? ids[r] : -1, r < end, pa);
     }
     __syncthreads();
     if (threadIdx.x < E) {                             // bases across chunks, totals
