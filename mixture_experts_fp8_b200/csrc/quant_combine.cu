@@ -17,62 +17,111 @@
 
 namespace moe {
 
-// One warp per (token, 128-column block).  Lane l owns columns 4l .. 4l+3 of the block.
+// One warp per (token, 512 columns): two 256-column chunks, both loads issued before any
+// arithmetic so that more bytes are in flight per warp.  In a chunk, lane l owns columns
+// 8l .. 8l+7 (one 16-byte load, one 8-byte code store per destination row): a 128-column group
+// is 16 lanes, a 32-column group 4 lanes.  H need only be a multiple of 128: lanes past the end
+// of the row take part in the shuffles but load and store nothing.
+constexpr int kQuantChunks = 2;
+
+__device__ __forceinline__ void quant_chunk(const QuantArgs& a, int t, int c, uint4 raw, bool in_row, int r_lane,
+                                            bool lane_row_ok) {
+    const int lane = threadIdx.x & 31;
+    float v[8];
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+        v[2 * i] = __low2float(b);
+        v[2 * i + 1] = __high2float(b);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    uint2 q;
+    float s32 = 1.0f;
+    uint8_t e8 = 127;
+    if (a.recipe == 0) {
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        s32 = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+        q.x = e4m3x4(__fdiv_rn(v[0], s32), __fdiv_rn(v[1], s32), __fdiv_rn(v[2], s32), __fdiv_rn(v[3], s32));
+        q.y = e4m3x4(__fdiv_rn(v[4], s32), __fdiv_rn(v[5], s32), __fdiv_rn(v[6], s32), __fdiv_rn(v[7], s32));
+    } else {
+#pragma unroll
+        for (int o = 1; o < 4; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const int e = mx_exponent(amax);
+        const float inv = exp2_int(-e);                 // x * 2^-e == x / 2^e exactly
+        q.x = e4m3x4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
+        q.y = e4m3x4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
+        e8 = static_cast<uint8_t>(e + 127);
+    }
+    const int A = a.T * a.K;
+    const int32_t* rows = a.row_of + static_cast<size_t>(t) * a.K;
+    const int col = c * 256 + 8 * lane;                // this lane's first column
+    const int g128 = col >> 7;                         // its 128-column block
+    for (int j = 0; j < a.K; ++j) {
+        const int r = j < 32 ? __shfl_sync(0xffffffffu, r_lane, j) : __ldg(rows + j);
+        if (r < 0 || r >= A) continue;                 // reported once per token by the caller
+        if (in_row) {
+            *reinterpret_cast<uint2*>(a.xq + static_cast<size_t>(r) * a.H + col) = q;
+            if (a.recipe != 0 && (lane & 3) == 0)
+                static_cast<uint8_t*>(a.xs)[(static_cast<size_t>(g128) * a.a_pad + r) * 4 + ((col >> 5) & 3)] = e8;
+        }
+    }
+    // fp32 scales, one per 128-column block: lane j stores block h's scale for the token's row j
+    if (a.recipe == 0) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float sh = __shfl_sync(0xffffffffu, s32, 16 * h);
+            const int gb = c * 2 + h;
+            if ((gb << 7) >= a.H) break;
+            if (lane < a.K && lane_row_ok) static_cast<float*>(a.xs)[static_cast<size_t>(gb) * a.a_pad + r_lane] = sh;
+            for (int j = 32 + lane; j < a.K; j += 32) {
+                const int r = __ldg(rows + j);
+                if (r >= 0 && r < A) static_cast<float*>(a.xs)[static_cast<size_t>(gb) * a.a_pad + r] = sh;
+            }
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
     pdl_wait_then_release();
     const int gw = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    const int nblk = a.H >> 7;
-    if (gw >= a.T * nblk) return;
-    const int t = gw / nblk, cb = gw - t * nblk;
-    const uint2 raw = *reinterpret_cast<const uint2*>(a.x + static_cast<size_t>(t) * a.H + cb * 128 + 4 * lane);
-    const __nv_bfloat162 p0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-    const __nv_bfloat162 p1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-    const float v0 = __low2float(p0), v1 = __high2float(p0), v2 = __low2float(p1), v3 = __high2float(p1);
-    float amax = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
-    uint32_t q;
-    float s32 = 1.0f;
-    uint8_t e8 = 127;
-    if (a.recipe == 0) {
-        amax = warp_max(amax);
-        s32 = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-        q = e4m3x4(__fdiv_rn(v0, s32), __fdiv_rn(v1, s32), __fdiv_rn(v2, s32), __fdiv_rn(v3, s32));
-    } else {
+    const int nchunks = (a.H + 255) >> 8;
+    const int nw = (nchunks + kQuantChunks - 1) / kQuantChunks;   // warps per token
+    if (gw >= a.T * nw) return;
+    const int t = gw / nw, c0 = (gw - t * nw) * kQuantChunks;
+    uint4 raw[kQuantChunks];
+    bool in_row[kQuantChunks];
 #pragma unroll
-        for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const int e = mx_exponent(amax);
-        const float inv = exp2_int(-e);                 // x * 2^-e == x / 2^e exactly
-        q = e4m3x4(v0 * inv, v1 * inv, v2 * inv, v3 * inv);
-        e8 = static_cast<uint8_t>(e + 127);
+    for (int i = 0; i < kQuantChunks; ++i) {
+        const int col = (c0 + i) * 256 + 8 * lane;
+        in_row[i] = c0 + i < nchunks && col < a.H;
+        raw[i] = in_row[i] ? __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.H + col))
+                           : make_uint4(0, 0, 0, 0);
     }
     // the token's destination rows: lane j holds row_of[t, j] (slots past 32 are read in the loop)
     const int A = a.T * a.K;
     const int32_t* rows = a.row_of + static_cast<size_t>(t) * a.K;
     const int r_lane = lane < a.K ? __ldg(rows + lane) : -1;
     const bool lane_row_ok = r_lane >= 0 && r_lane < A;
-    if (lane < a.K && !lane_row_ok) set_status(a.status, MOE_ERR_BOUNDS);
-    for (int j = 0; j < a.K; ++j) {
-        const int r = j < 32 ? __shfl_sync(0xffffffffu, r_lane, j) : __ldg(rows + j);
-        if (r < 0 || r >= A) {
-            if (j >= 32 && lane == 0) set_status(a.status, MOE_ERR_BOUNDS);
-            continue;
-        }
-        *reinterpret_cast<uint32_t*>(a.xq + static_cast<size_t>(r) * a.H + cb * 128 + 4 * lane) = q;
-        if (a.recipe != 0 && (lane & 7) == 0)
-            static_cast<uint8_t*>(a.xs)[(static_cast<size_t>(cb) * a.a_pad + r) * 4 + (lane >> 3)] = e8;
-    }
-    // fp32 scales: lane j stores the scale of the token's j-th row (one instruction for up to 32)
-    if (a.recipe == 0) {
-        if (lane < a.K && lane_row_ok) static_cast<float*>(a.xs)[static_cast<size_t>(cb) * a.a_pad + r_lane] = s32;
+    if (c0 == 0) {                                     // report a bad destination once per token
+        if (lane < a.K && !lane_row_ok) set_status(a.status, MOE_ERR_BOUNDS);
         for (int j = 32 + lane; j < a.K; j += 32) {
             const int r = __ldg(rows + j);
-            if (r >= 0 && r < A) static_cast<float*>(a.xs)[static_cast<size_t>(cb) * a.a_pad + r] = s32;
+            if (r < 0 || r >= A) set_status(a.status, MOE_ERR_BOUNDS);
         }
     }
+#pragma unroll
+    for (int i = 0; i < kQuantChunks; ++i)
+        if (c0 + i < nchunks) quant_chunk(a, t, c0 + i, raw[i], in_row[i], r_lane, lane_row_ok);
 }
 
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t s) {
-    const int warps = a.T * (a.H >> 7);
+    const int nchunks = (a.H + 255) >> 8;
+    const int warps = a.T * ((nchunks + kQuantChunks - 1) / kQuantChunks);
     return launch_pdl(k_quant, dim3((warps + 7) / 8), dim3(256), 0, s, a);
 }
 
@@ -83,10 +132,11 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
     __shared__ float s_w[MOE_MAX_EXPERTS + 1];
     pdl_wait_then_release();
     const int t = blockIdx.x;
-    const int A = a.T * a.K;
     for (int j = threadIdx.x; j < a.K; j += blockDim.x) {
-        int r = a.row_of[static_cast<size_t>(t) * a.K + j];
-        s_row[j] = (r >= 0 && r < A) ? r : 0;
+        const int r = a.row_of[static_cast<size_t>(t) * a.K + j];
+        const bool ok = r >= 0 && r < a.rows;
+        if (!ok && blockIdx.y == 0) set_status(a.status, MOE_ERR_BOUNDS);
+        s_row[j] = ok ? r : -1;
         s_w[j] = j < a.k ? a.w[static_cast<size_t>(t) * a.k + j] : 1.0f;   // shared expert: weight 1
     }
     __syncthreads();
@@ -94,6 +144,7 @@ __global__ void __launch_bounds__(256) k_combine(CombineArgs a) {
     if (c >= (a.H >> 2)) return;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < a.K; ++j) {
+        if (s_row[j] < 0) continue;                  // a position out of range adds nothing
         const float4 v = __ldg(reinterpret_cast<const float4*>(a.o + static_cast<size_t>(s_row[j]) * a.H) + c);
         const float w = s_w[j];
         acc.x = fmaf(w, v.x, acc.x);

@@ -95,6 +95,29 @@ def test_permutation_and_quantization(problems, name):
         assert np.array_equal(xs[rows], s_ref), f"scales differ (slot {j})"
 
 
+@pytest.mark.parametrize("hidden", [128, 384, 640, 896])
+@pytest.mark.parametrize("recipe", [0, 1])
+def test_quantization_odd_widths(hidden, recipe):
+    """Rows whose width is not a multiple of the quantizer's 256-column chunks (a half chunk at
+    the end), several chunk pairs per row, and more routed slots than a warp has lanes: every
+    permuted row's codes and scales bit for bit."""
+    shape = synth.Shape("q_odd", 37, hidden, 128, 48, 40, renormalize=1, recipe=recipe, seed=81)
+    prob = synth.make_problem(shape)
+    gp = GpuProblem(prob)
+    ni = oracle_inputs(prob)
+    idx, w, _ = oracle.route(oracle_cfg(shape), ni["logits"], None)
+    gp.forward(topk_idx=torch.from_numpy(idx).cuda(), topk_weights=torch.from_numpy(w).cuda())
+    assert gp.status() == 0
+    T, K, H = shape.num_tokens, shape.top_k, shape.hidden
+    _, _, _, row_of = oracle.permute(idx, shape.num_experts)
+    xq = gp.ws_region("xq", torch.uint8, T * K * H).cpu().numpy().reshape(T * K, H)
+    xs = gp.ws_scales("xs", H)
+    q_ref, s_ref = oracle.quantize_tokens(ni["x"], recipe)
+    for j in range(K):
+        assert np.array_equal(xq[row_of[:, j]], q_ref), f"codes differ (slot {j})"
+        assert np.array_equal(xs[row_of[:, j]], s_ref), f"scales differ (slot {j})"
+
+
 @pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "skewed", "large", "prefill_w4a8"])
 def test_gate_up_swiglu_codes(problems, name):
     """The gate+up GEMM's requantized SwiGLU products (E4M3 codes and scales) against the
