@@ -215,7 +215,7 @@ int moe_gate(const moe_config_t *cfg, const void *hidden_states, const void *gat
  *   y                 device bf16 [T, H], contiguous; out
  *   expert_counts     device int32 [E'] or NULL; out: rows routed to each expert (the shared
  *                     expert's count is num_tokens)
- *   workspace         device, >= moe_workspace_size bytes, 1024-byte aligned; scratch owned by
+ *   workspace         device, >= moe_workspace_size bytes, 256-byte aligned; scratch owned by
  *                     the caller; must not be shared by calls in flight at the same time
  * A row's output bits do not depend on the other rows of the batch. */
 int moe_forward(const moe_config_t *cfg, const void *hidden_states, const float *router_logits,
@@ -239,15 +239,38 @@ int moe_forward(const moe_config_t *cfg, const void *hidden_states, const float 
  *   device current; make that first call before any stream capture.  The array is shared by
  *   every call on the device and keeps the last call's contents (the forward clears its status
  *   word itself); calls that overlap on the GPU race on it.  Allocates nothing: no cudaMalloc,
- *   no cudaFree, no allocating library routine.  The status word (moe_read_status) lives in
- *   the array, so it cannot be read through this entry point's API; errors are still reported
- *   by the return code. */
+ *   no cudaFree, no allocating library routine.  The return code reports what the host checks
+ *   find and launch failures; faults the kernels find on the device (a bounded wait that ran
+ *   out, an index out of range) land in the array's status word, read with
+ *   moe_static_workspace_status. */
 int moe_forward_static_workspace(const moe_config_t *cfg, const void *hidden_states,
                                  const float *router_logits, const float *per_expert_scale,
                                  const int32_t *topk_idx, const float *topk_weights,
                                  const void *w13_t, const void *w13s_t, const void *w2_t,
                                  const void *w2s_t, const void *w13_bias, const void *w2_bias,
                                  void *y, int32_t *expert_counts, void *stream);
+
+/* Test hook, the gate+up step taken apart ("DeepGEMM PR #371", Testing: overlapped and
+ * non-overlapped runs give bitwise-identical outputs).  Runs the forward's permutation and
+ * quantization from the given routing, then the forward's gate+up GEMM kernel with its
+ * down-projection epilogue, storing the promoted fp32 gate/up sums without bias into h, then a
+ * separate SwiGLU + requantization kernel that writes the act codes and scales into the
+ * workspace (moe_workspace_layout: act_q, act_s), where moe_forward's fused epilogue writes them.
+ *   topk_idx          device int32 [T, k], ids in [0, E)
+ *   w13_t, w13s_t     as for moe_forward;  w13_bias device bf16 [E', 2I] or NULL
+ *   h                 device fp32 [T*(k + shared_experts), 2I], 32-byte aligned; out, columns in
+ *                     the transformed order of w13_t
+ *   workspace         as for moe_forward
+ * The codes and scales must equal moe_forward's bit for bit on the same inputs. */
+int moe_debug_unfused_gate_up(const moe_config_t *cfg, const void *hidden_states, const int32_t *topk_idx,
+                              const void *w13_t, const void *w13s_t, const void *w13_bias, float *h,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/* The status word of the last moe_forward_static_workspace call on the current device
+ * (MOE_OK, or MOE_ERR_TIMEOUT / MOE_ERR_BOUNDS set by a kernel), like moe_read_status: it
+ * synchronizes `stream`, then copies the word into *status (host).  The pages have no
+ * counterpart of this entry point. */
+int moe_static_workspace_status(int32_t *status, void *stream);
 
 /* moe_forward, recording a CUDA event before each of the MOE_NUM_STAGES stages and after the
  * last one into `prof` (which accumulates per-stage device time until reset).  prof may be
@@ -275,8 +298,9 @@ int moe_forward_profiled(const moe_config_t *cfg, const void *hidden_states,
  *   send_expert     device int32 [A]       out: each slot's expert id local to its destination
  *   slot_pos        device int32 [T, k]    out: each slot's position in send order
  *   workspace       as for moe_forward with the same cfg (scratch for the ordering)
- *   Four launches.  An expert id outside [0, E) is reported as MOE_ERR_BOUNDS in the workspace's
- *   status word (moe_read_status) and its slot is not sent.
+ *   A memset and four launches.  An expert id outside [0, E) is reported as MOE_ERR_BOUNDS in
+ *   the workspace's status word (moe_read_status); its slot is not sent (not counted in
+ *   send_counts) and its slot_pos is -1.
  *
  * The caller then exchanges send_x and send_expert (all-to-all with the counts: NCCL, or peer
  * copies), and every rank runs moe_forward_rows on the N rows it received:
@@ -296,7 +320,12 @@ int moe_forward_profiled(const moe_config_t *cfg, const void *hidden_states,
  *
  * moe_combine_rows: y[t] = bf16_rn( sum_j topk_weights[t,j] * o_home[slot_pos[t,j]] ), fp32, in
  * slot order: the combine of moe_forward, so y is bit-identical to the single-GPU forward.
- *   o_rows          device fp32 [T*k, H], 16-byte aligned;  y device bf16 [T, H], 16-byte aligned
+ *   o_rows          device fp32 [num_rows, H], 16-byte aligned (may be NULL when num_rows is 0)
+ *   num_rows        rows of o_rows: the sum of the send counts, in [0, T*k]
+ *   slot_pos        device int32 [T, k] from moe_ep_dispatch
+ *   y               device bf16 [T, H], 16-byte aligned; out
+ *   status          device int32 or NULL: a slot whose position lies outside [0, num_rows) adds
+ *                   nothing to its token's sum and sets it to MOE_ERR_BOUNDS (if it held MOE_OK)
  *   One launch. */
 int moe_ep_dispatch(const moe_config_t *cfg, int ranks, const void *hidden_states, const int32_t *topk_idx,
                     int32_t *send_counts, void *send_x, int32_t *send_expert, int32_t *slot_pos,
@@ -305,8 +334,8 @@ int moe_forward_rows(const moe_config_t *cfg, const void *rows, const int32_t *e
                      const void *w13_t, const void *w13s_t, const void *w2_t, const void *w2s_t,
                      const void *w13_bias, const void *w2_bias, float *o_rows, void *workspace,
                      size_t workspace_bytes, void *stream);
-int moe_combine_rows(const moe_config_t *cfg, const float *o_rows, const int32_t *slot_pos,
-                     const float *topk_weights, void *y, void *stream);
+int moe_combine_rows(const moe_config_t *cfg, const float *o_rows, int32_t num_rows, const int32_t *slot_pos,
+                     const float *topk_weights, void *y, int32_t *status, void *stream);
 
 /* Create / destroy a stage profiler (creates CUDA events on the current device). */
 int moe_profile_create(moe_profile_t **prof);

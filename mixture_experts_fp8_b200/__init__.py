@@ -34,7 +34,8 @@ EXPORTED = (
     "moe_last_error", "moe_check_config", "moe_transformed_weights_size", "moe_transform_weights",
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_forward", "moe_forward_profiled",
     "moe_profile_create", "moe_profile_destroy", "moe_profile_read", "moe_profile_reset",
-    "moe_read_status", "moe_selftest_bounded_wait", "moe_forward_static_workspace",
+    "moe_read_status", "moe_selftest_bounded_wait", "moe_forward_static_workspace", "moe_static_workspace_status",
+    "moe_debug_unfused_gate_up",
     "moe_debug_inject_fault", "moe_gate", "moe_gate_weights_size", "moe_transform_gate_weights",
     "moe_ep_dispatch", "moe_forward_rows", "moe_combine_rows",
 )
@@ -132,13 +133,15 @@ def _load():
             "moe_read_status": [P, P, P],
             "moe_selftest_bounded_wait": [P, ctypes.c_uint32, P],
             "moe_forward_static_workspace": [CP] + [P] * 13 + [P],
+            "moe_static_workspace_status": [P, P],
+            "moe_debug_unfused_gate_up": [CP] + [P] * 7 + [S, P],
             "moe_debug_inject_fault": [I],
             "moe_gate": [CP, P, P, ctypes.c_float, P, P, P, P, P],
             "moe_gate_weights_size": [CP, ctypes.POINTER(S)],
             "moe_transform_gate_weights": [CP, P, P, P, P],
             "moe_ep_dispatch": [CP, I, P, P, P, P, P, P, P, S, P],
             "moe_forward_rows": [CP] + [P] * 10 + [S, P],
-            "moe_combine_rows": [CP, P, P, P, P, P],
+            "moe_combine_rows": [CP, P, ctypes.c_int32, P, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(lib, name)
@@ -301,15 +304,18 @@ def forward_rows(cfg: Config, rows, expert_of_row, weights, w13_bias=None, w2_bi
     return o_rows
 
 
-def combine_rows(cfg: Config, o_rows, slot_pos, topk_weights, y=None, stream=None):
-    """y[t] = bf16(sum_j w[t,j] * o_rows[slot_pos[t,j]]) in slot order -> y bf16 [T, H]."""
+def combine_rows(cfg: Config, o_rows, slot_pos, topk_weights, y=None, status=None, stream=None):
+    """y[t] = bf16(sum_j w[t,j] * o_rows[slot_pos[t,j]]) in slot order -> y bf16 [T, H].  A slot
+    whose position is outside o_rows adds nothing and sets `status` (device int32) to
+    MOE_ERR_BOUNDS."""
     import torch
     T, H = cfg.num_tokens, cfg.hidden
     if y is None:
-        y = torch.empty((T, H), dtype=torch.bfloat16, device=o_rows.device)
+        y = torch.empty((T, H), dtype=torch.bfloat16, device=slot_pos.device)
     c = cfg.c()
-    _check(_load().moe_combine_rows(ctypes.byref(c), _ptr(o_rows), _ptr(slot_pos), _ptr(topk_weights), _ptr(y),
-                                    _stream(stream)))
+    n = int(o_rows.shape[0])
+    _check(_load().moe_combine_rows(ctypes.byref(c), _ptr(o_rows) if n else None, n, _ptr(slot_pos),
+                                    _ptr(topk_weights), _ptr(y), _ptr(status), _stream(stream)))
     return y
 
 
@@ -355,6 +361,28 @@ def forward_static_workspace(cfg: Config, hidden_states, weights, router_logits=
 def read_status(workspace, stream=None) -> int:
     st = ctypes.c_int32()
     _check(_load().moe_read_status(_ptr(workspace), ctypes.byref(st), _stream(stream)))
+    return st.value
+
+
+def debug_unfused_gate_up(cfg: Config, hidden_states, topk_idx, weights, workspace, w13_bias=None, stream=None):
+    """The gate+up step taken apart (test hook): the GEMM stores the fp32 gate/up sums h, then a
+    separate SwiGLU + requantization kernel writes the act codes and scales into `workspace`.
+    Returns h [A, 2I] fp32 (columns in the transformed order)."""
+    import torch
+    A = cfg.num_tokens * (cfg.top_k + cfg.shared_experts)
+    h = torch.empty((A, 2 * cfg.inter), dtype=torch.float32, device=hidden_states.device)
+    c = cfg.c()
+    w13_t, w13s_t = weights[0], weights[1]
+    _check(_load().moe_debug_unfused_gate_up(ctypes.byref(c), _ptr(hidden_states), _ptr(topk_idx), _ptr(w13_t),
+                                             _ptr(w13s_t), _ptr(w13_bias), _ptr(h), _ptr(workspace),
+                                             workspace.numel(), _stream(stream)))
+    return h
+
+
+def static_workspace_status(stream=None) -> int:
+    """The status word of the last moe_forward_static_workspace call on the current device."""
+    st = ctypes.c_int32()
+    _check(_load().moe_static_workspace_status(ctypes.byref(st), _stream(stream)))
     return st.value
 
 

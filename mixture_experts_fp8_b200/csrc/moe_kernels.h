@@ -83,11 +83,13 @@ struct QuantArgs {
 };
 
 struct CombineArgs {
-    const float* o;             // [A, H]
+    const float* o;             // [rows, H]
     const int32_t* row_of;      // [T, K]  (K slots per token)
     const float* w;             // [T, k]  routing weights of the k routed slots
     __nv_bfloat16* y;           // [T, H]
     int T, H, K, k;             // slots j >= k (the shared expert's) have weight 1
+    int rows;                   // rows of o: a slot whose position is outside [0, rows) adds nothing
+    int32_t* status;            // and is reported here as MOE_ERR_BOUNDS (when non-null)
 };
 
 // Expert parallelism (ep.cu): slot i = t * K + j of this rank's routing.
@@ -145,6 +147,7 @@ cudaError_t launch_rows_f32(const float* o, const int32_t* row_of, float* out, i
 uint32_t gemm_weight_box(int mode);
 cudaError_t launch_gemm(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB,
                         int num_sms, cudaStream_t s);
+
 cudaError_t launch_gemm_mx(const GemmArgs& a, const CUtensorMap& tmA, const CUtensorMap& tmB, int num_sms,
                            cudaStream_t s);
 cudaError_t launch_gemm_mx_narrow(const GemmArgs& a, const CUtensorMap& tmW, const CUtensorMap& tmT, int num_sms,
@@ -154,6 +157,10 @@ cudaError_t launch_gemm_narrow(const GemmArgs& a, const CUtensorMap& tmW, const 
                                int num_sms, cudaStream_t s);
 // The narrow (swap-AB) GEMMs take problems averaging at most this many routed rows per expert.
 constexpr int kNarrowRowsPerExpert = 32;
+// The SwiGLU + requantization step on its own (unfused.cu): h [A, 2I] fp32 in the transformed
+// column order -> act codes and scales, as the gate+up epilogue computes them.
+cudaError_t launch_swiglu_requant(const float* h, const __nv_bfloat16* bias, const int32_t* offsets, uint8_t* act_q,
+                                  void* act_s, int A, int I, int E, int recipe, int a_pad, cudaStream_t s);
 int set_last_error(int code, const char* msg);
 cudaError_t launch_selftest_wait(int32_t* status, uint32_t timeout_us, cudaStream_t s);
 

@@ -96,6 +96,8 @@ int take_armed_fault() {
     return f;
 }
 
+// Rows of the stage-major activation scales: every routed row, plus the reach of the last GEMM
+// tile's 16-byte-aligned scale run (132 words from its first row rounded down to 4).
 size_t scale_rows_of(size_t A) { return align_up(A + moe::kTileM + 4, 4); }
 
 void layout_of(const moe_config_t* c, moe_workspace_layout_t* L) {
@@ -434,7 +436,7 @@ int forward_impl(const moe_config_t* cfg, const void* hidden_states, const float
                                           static_cast<const int32_t*>(at(L.row_of)), o_rows, T, H, status, s));
     } else {
         moe::CombineArgs ca{static_cast<const float*>(at(L.o)), static_cast<const int32_t*>(at(L.row_of)), wts,
-                            static_cast<__nv_bfloat16*>(y), T, H, KT, K};
+                            static_cast<__nv_bfloat16*>(y), T, H, KT, K, A, status};
         MOE_CUDA_TRY(moe::launch_combine(ca, s));
     }
     MOE_CUDA_TRY(mark(6));
@@ -475,6 +477,78 @@ int moe_forward_rows(const moe_config_t* cfg, const void* rows, const int32_t* e
                         w2_bias, nullptr, o_rows, nullptr, workspace, workspace_bytes, nullptr, stream);
 }
 
+int moe_debug_unfused_gate_up(const moe_config_t* cfg, const void* hidden_states, const int32_t* topk_idx,
+                              const void* w13_t, const void* w13s_t, const void* w13_bias, float* h,
+                              void* workspace, size_t workspace_bytes, void* stream_) {
+    int rc = check_config(cfg);
+    if (rc) return rc;
+    if (!hidden_states || !topk_idx || !w13_t || !w13s_t || !h || !workspace)
+        return fail(MOE_ERR_INVALID_ARG, "moe_debug_unfused_gate_up: NULL pointer");
+    if (!aligned(hidden_states, 16) || !aligned(topk_idx, 4) || !aligned(w13_t, 32) || !aligned(w13s_t, 16) ||
+        !aligned(h, 32) || !aligned(workspace, 256) || (w13_bias && !aligned(w13_bias, 16)))
+        return fail(MOE_ERR_INVALID_ARG, "moe_debug_unfused_gate_up: misaligned buffer");
+    moe_workspace_layout_t L;
+    layout_of(cfg, &L);
+    if (workspace_bytes < L.total)
+        return fail(MOE_ERR_INVALID_ARG, "moe_debug_unfused_gate_up: workspace has %zu bytes, needs %zu",
+                    workspace_bytes, L.total);
+    DeviceInfo di;
+    if ((rc = device_info(&di))) return rc;
+    const int T = cfg->num_tokens, K = cfg->top_k, E = cfg->num_experts, H = cfg->hidden, I = cfg->inter;
+    const int KT = K + cfg->shared_experts, ET = E + cfg->shared_experts;
+    const int A = T * KT;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto at = [&](size_t off) { return static_cast<void*>(ws + off); };
+    int32_t* status = static_cast<int32_t*>(at(L.status));
+    // the forward's choice of GEMM kernel and tensor-map boxes (see forward_impl)
+    const bool mx = cfg->recipe != 0;
+    const bool fp4 = cfg->recipe == 2;
+    const bool narrow = A <= moe::kNarrowRowsPerExpert * ET;
+    CUtensorMap tm_x, tm_w13;
+    const uint32_t tok_box = !narrow ? moe::kTileM : mx ? moe::gemm_mx_narrow_tokens() : 16;
+    const uint32_t w13_box = mx ? 128 : narrow ? moe::kTileN : moe::gemm_weight_box(0);
+    if ((rc = make_kmajor_map(&tm_x, at(L.xq), A, H, tok_box))) return rc;
+    if ((rc = make_kmajor_map(&tm_w13, w13_t, static_cast<uint64_t>(ET) * 2 * I, H, w13_box, fp4))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream_);
+    MOE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    moe::PermuteArgs pa{topk_idx, static_cast<int32_t*>(at(L.hist)), static_cast<int32_t*>(at(L.counts)),
+                        static_cast<int32_t*>(at(L.offsets)), static_cast<int32_t*>(at(L.tile_start)),
+                        static_cast<int32_t*>(at(L.row_src)), static_cast<int32_t*>(at(L.row_of)), nullptr,
+                        status, A, E, moe::permute_chunks(A), moe::permute_chunk_rows(A), T, K, KT};
+    if (A <= moe::kSmallRows) MOE_CUDA_TRY(moe::launch_permute_small(pa, false, s));
+    else MOE_CUDA_TRY(moe::launch_permute(pa, s));
+    moe::QuantArgs qa{static_cast<const __nv_bfloat16*>(hidden_states), static_cast<const int32_t*>(at(L.row_of)),
+                      static_cast<uint8_t*>(at(L.xq)), at(L.xs), status, T, H, KT, cfg->recipe,
+                      static_cast<int>(L.scale_rows)};
+    MOE_CUDA_TRY(moe::launch_quant(qa, s));
+    // GEMM1 with the down projection's epilogue: h = the promoted gate/up sums, fp32, no bias
+    moe::GemmArgs g{};
+    g.mode = 1;
+    g.recipe = cfg->recipe;
+    g.N = 2 * I;
+    g.K = H;
+    g.E = ET;
+    g.A = A;
+    g.a_pad = static_cast<int>(L.scale_rows);
+    g.offsets = static_cast<const int32_t*>(at(L.offsets));
+    g.tile_start = static_cast<const int32_t*>(at(L.tile_start));
+    g.a_scale = at(L.xs);
+    g.w_scale = w13s_t;
+    g.bias = nullptr;
+    g.out = h;
+    g.status = status;
+    g.fault = MOE_FAULT_NONE;
+    MOE_CUDA_TRY(mx ? (narrow ? moe::launch_gemm_mx_narrow(g, tm_w13, tm_x, di.sms, s)
+                              : moe::launch_gemm_mx(g, tm_x, tm_w13, di.sms, s))
+                    : (narrow ? moe::launch_gemm_narrow(g, tm_w13, tm_x, di.sms, s)
+                              : moe::launch_gemm(g, tm_x, tm_w13, di.sms, s)));
+    MOE_CUDA_TRY(moe::launch_swiglu_requant(h, static_cast<const __nv_bfloat16*>(w13_bias),
+                                            static_cast<const int32_t*>(at(L.offsets)),
+                                            static_cast<uint8_t*>(at(L.act_q)), at(L.act_s), A, I, ET, cfg->recipe,
+                                            static_cast<int>(L.scale_rows), s));
+    return ok();
+}
+
 int moe_ep_dispatch(const moe_config_t* cfg, int ranks, const void* hidden_states, const int32_t* topk_idx,
                     int32_t* send_counts, void* send_x, int32_t* send_expert, int32_t* slot_pos, void* workspace,
                     size_t workspace_bytes, void* stream_) {
@@ -502,6 +576,8 @@ int moe_ep_dispatch(const moe_config_t* cfg, int ranks, const void* hidden_state
     int32_t* row_src = static_cast<int32_t*>(at(L.row_src));
     cudaStream_t s = static_cast<cudaStream_t>(stream_);
     MOE_CUDA_TRY(cudaMemsetAsync(status, 0, sizeof(int32_t), s));
+    // a slot that is not sent (an expert id out of range) keeps position -1
+    MOE_CUDA_TRY(cudaMemsetAsync(slot_pos, 0xFF, sizeof(int32_t) * static_cast<size_t>(A), s));
     moe::EpArgs ea{topk_idx, dest, row_src, static_cast<const __nv_bfloat16*>(hidden_states),
                    static_cast<__nv_bfloat16*>(send_x), send_expert, status, A, K, cfg->hidden, E, E / ranks};
     MOE_CUDA_TRY(moe::launch_ep_dest(ea, s));
@@ -516,19 +592,23 @@ int moe_ep_dispatch(const moe_config_t* cfg, int ranks, const void* hidden_state
     return ok();
 }
 
-int moe_combine_rows(const moe_config_t* cfg, const float* o_rows, const int32_t* slot_pos,
-                     const float* topk_weights, void* y, void* stream) {
+int moe_combine_rows(const moe_config_t* cfg, const float* o_rows, int32_t num_rows, const int32_t* slot_pos,
+                     const float* topk_weights, void* y, int32_t* status, void* stream) {
     int rc = check_config(cfg);
     if (rc) return rc;
     if (cfg->shared_experts != 0)
         return fail(MOE_ERR_UNSUPPORTED, "moe_combine_rows: expert parallelism takes no shared expert");
-    if (!o_rows || !slot_pos || !topk_weights || !y) return fail(MOE_ERR_INVALID_ARG, "moe_combine_rows: NULL pointer");
-    if (!aligned(o_rows, 16) || !aligned(y, 16) || !aligned(slot_pos, 4) || !aligned(topk_weights, 4))
+    if (num_rows < 0 || static_cast<long long>(num_rows) > static_cast<long long>(cfg->num_tokens) * cfg->top_k)
+        return fail(MOE_ERR_INVALID_ARG, "moe_combine_rows: num_rows %d outside [0, T*k]", num_rows);
+    if ((!o_rows && num_rows > 0) || !slot_pos || !topk_weights || !y)
+        return fail(MOE_ERR_INVALID_ARG, "moe_combine_rows: NULL pointer");
+    if (!aligned(o_rows, 16) || !aligned(y, 16) || !aligned(slot_pos, 4) || !aligned(topk_weights, 4) ||
+        !aligned(status, 4))
         return fail(MOE_ERR_INVALID_ARG, "moe_combine_rows: misaligned buffer (rows need 16 bytes)");
     DeviceInfo di;
     if ((rc = device_info(&di))) return rc;
     moe::CombineArgs ca{o_rows, slot_pos, topk_weights, static_cast<__nv_bfloat16*>(y), cfg->num_tokens, cfg->hidden,
-                        cfg->top_k, cfg->top_k};
+                        cfg->top_k, cfg->top_k, num_rows, status};
     MOE_CUDA_TRY(moe::launch_combine(ca, static_cast<cudaStream_t>(stream)));
     return ok();
 }

@@ -15,7 +15,9 @@
 // stream capture begins.  All calls on a device share the array and it keeps the last call's
 // contents; the forward clears what must start at zero (its status word) itself.  Calls that
 // overlap on the GPU (different streams, or different host threads, without ordering between
-// them) race on the array and corrupt each other's results.
+// them) race on the array and corrupt each other's results.  Faults the kernels find on the
+// device (a bounded wait that ran out, an index out of range) land in the array's status word;
+// moe_static_workspace_status reads it.
 #include <cstdio>
 #include <mutex>
 
@@ -31,6 +33,29 @@ __device__ __align__(256) uint8_t g_static_workspace[kStaticWorkspaceBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_ws_addr[kMaxDevices] = {nullptr};
+
+// The device address of the array on the current device (looked up once per device).
+int static_ws_addr(const char* who, void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return moe::set_last_error(MOE_ERR_CUDA, cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) {
+        char msg[160];
+        snprintf(msg, sizeof(msg), "%s: device ordinal out of range", who);
+        return moe::set_last_error(MOE_ERR_UNSUPPORTED, msg);
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_ws_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_workspace);
+        if (e != cudaSuccess || !p)
+            return moe::set_last_error(MOE_ERR_CUDA, e != cudaSuccess ? cudaGetErrorString(e)
+                                                                        : "cudaGetSymbolAddress returned NULL");
+        g_ws_addr[dev] = p;
+    }
+    *out = g_ws_addr[dev];
+    return MOE_OK;
+}
 
 }  // namespace
 
@@ -53,27 +78,21 @@ int moe_forward_static_workspace(const moe_config_t* cfg, const void* hidden_sta
                  need, kStaticWorkspaceBytes);
         return moe::set_last_error(MOE_ERR_UNSUPPORTED, msg);
     }
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return moe::set_last_error(MOE_ERR_CUDA, cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices)
-        return moe::set_last_error(MOE_ERR_UNSUPPORTED, "moe_forward_static_workspace: device ordinal out of range");
     void* ws = nullptr;
-    {
-        std::lock_guard<std::mutex> lock(g_mu);
-        if (!g_ws_addr[dev]) {
-            void* p = nullptr;
-            e = cudaGetSymbolAddress(&p, g_static_workspace);
-            if (e != cudaSuccess || !p)
-                return moe::set_last_error(MOE_ERR_CUDA, e != cudaSuccess ? cudaGetErrorString(e)
-                                                                            : "cudaGetSymbolAddress returned NULL");
-            g_ws_addr[dev] = p;
-        }
-        ws = g_ws_addr[dev];
-    }
+    if ((rc = static_ws_addr("moe_forward_static_workspace", &ws)) != MOE_OK) return rc;
     return moe_forward(cfg, hidden_states, router_logits, per_expert_scale, topk_idx, topk_weights, w13_t,
                        w13s_t, w2_t, w2s_t, w13_bias, w2_bias, y, expert_counts, ws, kStaticWorkspaceBytes,
                        stream);
+}
+
+// The status word of the last forward run through the array (it sits at the start of every
+// workspace): after synchronizing `stream`, a blocking 4-byte copy, like moe_read_status.
+int moe_static_workspace_status(int32_t* status, void* stream) {
+    if (!status) return moe::set_last_error(MOE_ERR_INVALID_ARG, "moe_static_workspace_status: NULL status");
+    void* ws = nullptr;
+    const int rc = static_ws_addr("moe_static_workspace_status", &ws);
+    if (rc != MOE_OK) return rc;
+    return moe_read_status(ws, status, stream);
 }
 
 }  // extern "C"

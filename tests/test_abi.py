@@ -169,7 +169,9 @@ def test_expert_parallel_entry_points_validate_before_any_cuda_call():
     one = cfg(num_experts=4, top_k=1).c()
     rc = lib.moe_forward_rows(ctypes.byref(one), al, None, al, al, al, al, None, None, al, al, 1 << 20, None)
     assert rc == moe.MOE_ERR_INVALID_ARG and b"NULL" in lib.moe_last_error()
-    rc = lib.moe_combine_rows(ctypes.byref(c), al, None, al, al, None)
+    rc = lib.moe_combine_rows(ctypes.byref(c), al, 4, None, al, al, None, None)
     assert rc == moe.MOE_ERR_INVALID_ARG and b"NULL" in lib.moe_last_error()
-    rc = lib.moe_combine_rows(ctypes.byref(c), al | 4, al, al, al, None)
+    rc = lib.moe_combine_rows(ctypes.byref(c), al | 4, 4, al, al, al, None, None)
     assert rc == moe.MOE_ERR_INVALID_ARG and b"misaligned" in lib.moe_last_error()
+    rc = lib.moe_combine_rows(ctypes.byref(c), al, 1 << 30, al, al, al, None, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG and b"num_rows" in lib.moe_last_error()

@@ -4,11 +4,18 @@ Some callers run inside a host framework that owns every byte of device memory (
 engine's pre-reserved pool, or a plugin interface that hands its kernels no scratch buffer);
 they cannot call cudaMalloc, which can synchronize the device and can fail under memory pressure.
 This entry point takes the same inputs and outputs as moe_forward but keeps its scratch in a
-fixed 16 MiB array inside the library.  Its output must match moe_forward's (same kernels) within
-the tolerance the other parity tests use, on two calls in a row (the array keeps the previous
-call's contents).  This file is named to be collected last, and passes alone or after the rest.
+fixed 16 MiB array inside the library.  It runs the same kernels on the same inputs, so its
+output must equal moe_forward's bit for bit, on two calls in a row (the array keeps the previous
+call's contents).  Faults found on the device land in the array's status word, which
+moe_static_workspace_status reads: a stage dropped on purpose by the debug library (in a child
+process) must read back as a timeout, and the next call must be clean.  This file is named to be
+collected last, and passes alone or after the rest.
 """
 import ctypes
+import json
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -16,9 +23,11 @@ import torch
 
 import mixture_experts_fp8_b200 as moe
 import synth
-from _helpers import GpuProblem, assert_y_close, bits
+from _helpers import GpuProblem, bits
 
 pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _call(gp, y):
@@ -41,7 +50,8 @@ def test_static_workspace_matches_moe_forward_twice(name):
     for _ in range(2):
         y = torch.full((gp.shape.num_tokens, gp.shape.hidden), float("nan"), dtype=torch.bfloat16, device="cuda")
         assert _call(gp, y) == moe.MOE_OK, moe.lib().moe_last_error()
-        assert_y_close(bits(y), ref, f"{name} static workspace")
+        assert np.array_equal(bits(y), ref), f"{name}: static workspace output differs from moe_forward"
+        assert moe.static_workspace_status() == moe.MOE_OK
 
 
 def test_static_workspace_rejects_problems_that_do_not_fit():
@@ -52,3 +62,32 @@ def test_static_workspace_rejects_problems_that_do_not_fit():
     rc = moe.lib().moe_forward_static_workspace(ctypes.byref(c), *([ctypes.c_void_p(16)] * 13), None)
     assert rc == moe.MOE_ERR_UNSUPPORTED
     assert b"16777216" in moe.lib().moe_last_error()
+
+
+CHILD = r"""
+import ctypes, json, sys, numpy as np, torch
+sys.path.insert(0, ROOT); sys.path.insert(0, ROOT + "/tests")
+import mixture_experts_fp8_b200 as moe
+from mixture_experts_fp8_b200 import build as b
+moe.LIB_PATH = b.build(debug=True)
+import synth
+from _helpers import GpuProblem, bits
+from test_zz_no_alloc import _call
+gp = GpuProblem(synth.make_problem("tiny"))
+y = torch.empty((gp.shape.num_tokens, gp.shape.hidden), dtype=torch.bfloat16, device="cuda")
+moe.debug_inject_fault(moe.MOE_FAULT_SKIP_STAGE)
+rc1 = _call(gp, y); s1 = moe.static_workspace_status()
+rc2 = _call(gp, y); s2 = moe.static_workspace_status()
+same = bool(np.array_equal(bits(y), bits(gp.forward())))
+print(json.dumps([rc1, s1, rc2, s2, same]))
+"""
+
+
+def test_static_workspace_status_reports_a_device_fault():
+    code = f"ROOT = {ROOT!r}\n" + CHILD
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-3000:]
+    rc1, s1, rc2, s2, same = json.loads(r.stdout.strip().splitlines()[-1])
+    assert rc1 == moe.MOE_OK                   # the launch itself succeeded
+    assert s1 == moe.MOE_ERR_TIMEOUT           # the dropped stage is reported through the array
+    assert rc2 == moe.MOE_OK and s2 == moe.MOE_OK and same   # the next call is clean and exact
