@@ -47,11 +47,16 @@ class LibraryOps:
         return self.moe.forward_rows(cfg_rows, rows, expert_of_row, weights_local, w13_bias=w13_bias,
                                      w2_bias=w2_bias)
 
-    def combine(self, cfg, o_rows, slot_pos, topk_weights):
-        return self.moe.combine_rows(cfg, o_rows, slot_pos, topk_weights)
+    def combine(self, cfg, o_rows, slot_pos, topk_weights, status=None):
+        return self.moe.combine_rows(cfg, o_rows, slot_pos, topk_weights, status=status)
 
     def new_workspace(self, cfg, device):
         return self.moe.new_workspace(cfg, device)
+
+    def status_word(self, workspace):
+        """The dispatch's status word (device int32 [1]: the first word of the workspace)."""
+        import torch
+        return workspace[:4].view(torch.int32)
 
 
 def rows_config(cfg, ranks: int, n_rows: int):
@@ -90,8 +95,11 @@ def ep_step(cfg, ranks: int, x, router_logits, weights_local, dist, group=None, 
     sc = send_counts.to(torch.int64)
     rc = torch.empty_like(sc)
     dist.all_to_all_single(rc, sc, group=group)
-    both = torch.stack([sc, rc]).tolist()          # one read-back of both split lists
-    send_splits, recv_splits = [int(v) for v in both[0]], [int(v) for v in both[1]]
+    status = ops.status_word(workspace) if hasattr(ops, "status_word") else None
+    parts = [sc, rc] + ([status.to(torch.int64)] if status is not None else [])
+    vals = [int(v) for v in torch.cat(parts).tolist()]   # one read-back: both split lists, the status
+    send_splits, recv_splits = vals[:ranks], vals[ranks:2 * ranks]
+    dispatch_status = vals[2 * ranks] if status is not None else 0
     recv_x = all_to_all_rows(dist, group, send_x[:sum(send_splits)], send_splits, recv_splits)
     recv_e = all_to_all_rows(dist, group, send_expert[:sum(send_splits)], send_splits, recv_splits)
 
@@ -102,5 +110,11 @@ def ep_step(cfg, ranks: int, x, router_logits, weights_local, dist, group=None, 
     else:                              # nothing routed to this rank's experts
         o_recv = torch.empty((0, cfg.hidden), dtype=getattr(torch, ops.rows_dtype), device=dev)
     o_home = all_to_all_rows(dist, group, o_recv, recv_splits, send_splits)
-    y = ops.combine(cfg, o_home, slot_pos, w)
+    y = ops.combine(cfg, o_home, slot_pos, w, status=status)
+    if dispatch_status != 0:
+        # every rank has taken the same collective steps; only now report the bad routing (a slot
+        # whose expert id was out of range was not sent, and its token lacks that slot's term)
+        from . import MoeError
+        raise MoeError(dispatch_status, "moe_ep_dispatch: an expert id outside [0, num_experts) "
+                                        "(status word MOE_ERR_BOUNDS); its slot was not sent")
     return y, {"sent": send_splits, "received": recv_splits}

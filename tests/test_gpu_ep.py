@@ -4,15 +4,19 @@ destination rank.  Then R ranks are emulated in one process: each routes its own
 dispatches them, the all-to-all is a copy of row blocks on the device, each computes the rows it
 received with its own experts' weights, the rows go back, and each combines.  Every rank's y must
 equal the single-GPU forward of the whole problem on those tokens, bit for bit (a row's result
-depends only on its own codes and its expert's weights).  No kernel waits on another: the ranks
-run one after the other."""
+depends only on its own codes and its expert's weights), and must match the oracle's forward of
+those tokens within the layer's tolerance; each rank's expert-side rows must match the oracle's
+expert_rows on the rows it received.  No kernel waits on another: the ranks run one after the
+other.  An expert id out of range is reported, not sent, and adds nothing in the combine."""
 from dataclasses import replace
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
+from _helpers import Y_MAX_REL_RMS, Y_MEAN_REL, assert_y_close, bits, oracle_y
 
 pytestmark = pytest.mark.gpu
 
@@ -78,6 +82,7 @@ def _emulate(shape, ranks):
         assert moe.read_status(ws) == moe.MOE_OK
         plans.append(dict(w=w, counts=counts.cpu().tolist(), send_x=send_x, send_e=send_e, slot_pos=slot_pos))
     starts = [np.concatenate([[0], np.cumsum(p["counts"])]) for p in plans]
+    sides = []                                                 # (rank, rows, local ids, o) per expert side
     o_back = [torch.empty((T * shape.top_k, shape.hidden), dtype=torch.float32, device="cuda") for _ in plans]
     for q in range(ranks):                                     # each rank: the rows sent to it
         blocks = [(r, int(starts[r][q]), int(starts[r][q + 1])) for r in range(ranks)]
@@ -97,6 +102,7 @@ def _emulate(shape, ranks):
                              w2_bias=None if d.w2_bias is None else d.w2_bias[es].contiguous(), workspace=ws_q)
         torch.cuda.synchronize()
         assert moe.read_status(ws_q) == moe.MOE_OK
+        sides.append((q, rows, rows_e, o))
         off = 0
         for r, a, b in blocks:                                 # back to the senders' positions
             o_back[r][a:b] = o[off:off + (b - a)]
@@ -105,14 +111,68 @@ def _emulate(shape, ranks):
     for r in range(ranks):                                     # each rank: combine
         ys.append(moe.combine_rows(cfg, o_back[r], plans[r]["slot_pos"], plans[r]["w"]))
     torch.cuda.synchronize()
-    return torch.cat(ys), y_ref
+    return torch.cat(ys), y_ref, prob, sides
 
 
 @pytest.mark.parametrize("name,ranks", [("tiny_r0", 1), ("tiny_r0", 2), ("groups_mx", 4), ("w4a8", 2),
                                         ("decode", 2), ("decode", 8)])
 def test_emulated_ranks_match_the_single_gpu_forward(name, ranks):
-    y, y_ref = _emulate(SHAPES[name], ranks)
+    y, y_ref, _, _ = _emulate(SHAPES[name], ranks)
     assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+
+
+@pytest.mark.parametrize("name,ranks", [("tiny_r0", 2), ("groups_mx", 4), ("w4a8", 2), ("decode", 8)])
+def test_emulated_ranks_match_the_oracle(name, ranks):
+    """Every rank's y against the oracle's forward of the same tokens, and every expert side's
+    rows against the oracle's expert_rows on the rows that rank received."""
+    shape = SHAPES[name]
+    y, _, prob, sides = _emulate(shape, ranks)
+    ni = prob.numpy_inputs()
+    assert_y_close(bits(y), oracle_y(prob, ni), f"{name} over {ranks} ranks")
+    E_loc = shape.num_experts // ranks
+    ocfg = oracle.Config(**shape.cfg())
+    for q, rows, rows_e, o in sides:
+        es = slice(q * E_loc, (q + 1) * E_loc)
+        c = replace(ocfg, num_tokens=int(rows.shape[0]), top_k=1, num_experts=E_loc, routing=0, renormalize=0,
+               group_count=1, k_group=1, group_select_mode=0, routed_scaling_factor=1.0)
+        ref = oracle.expert_rows(c, rows.view(torch.int16).cpu().numpy().view(np.uint16), rows_e.cpu().numpy(),
+                                 ni["w13"][es], ni["w13s"][es], ni["w2"][es], ni["w2s"][es],
+                                 None if ni["b13"] is None else ni["b13"][es],
+                                 None if ni["b2"] is None else ni["b2"][es])
+        got = o.double().cpu().numpy()
+        d = np.abs(got - ref)
+        rms = float(np.sqrt(np.mean(ref * ref)))
+        assert d.max() <= Y_MAX_REL_RMS * rms, (name, q, d.max() / rms)
+        assert d.sum() / np.abs(ref).sum() <= Y_MEAN_REL, (name, q)
+
+
+def test_out_of_range_expert_is_reported_not_sent_and_adds_nothing():
+    """An expert id outside [0, E): the dispatch reports MOE_ERR_BOUNDS, does not send the slot and
+    leaves its position at -1; the combine over the rows that did come back adds nothing for it
+    and reports it in the status word it is given."""
+    moe = _lib()
+    shape = SHAPES["tiny_r0"]
+    d = synth.make_problem(shape).to("cuda")
+    cfg = moe.Config(**shape.cfg())
+    ws = moe.new_workspace(cfg, "cuda")
+    idx, w = moe.route(cfg, d.logits)
+    idx[3, 1] = shape.num_experts + 5                          # token 3, slot 1: no such expert
+    counts, send_x, send_e, slot_pos = moe.ep_dispatch(cfg, 2, d.x, idx, ws)
+    torch.cuda.synchronize()
+    assert moe.read_status(ws) == moe.MOE_ERR_BOUNDS
+    A = shape.num_tokens * shape.top_k
+    assert int(counts.sum()) == A - 1
+    assert int(slot_pos[3, 1]) == -1
+    n = A - 1
+    o = torch.ones((n, shape.hidden), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    w1 = torch.ones_like(w)
+    y = moe.combine_rows(cfg, o, slot_pos, w1, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == moe.MOE_ERR_BOUNDS
+    yf = y.float().cpu()
+    assert torch.all(yf[3] == 1.0)                             # only slot 0's row of ones
+    assert torch.all(yf[torch.arange(shape.num_tokens) != 3] == float(shape.top_k))
 
 
 def test_forward_rows_rejects_more_than_one_slot():

@@ -84,7 +84,7 @@ class OracleOps:
         o = oracle.expert_rows(_ocfg(cfg_rows), x, expert_of_row.numpy(), *weights_local, b13, b2)
         return torch.from_numpy(o)
 
-    def combine(self, cfg, o_rows, slot_pos, topk_weights):
+    def combine(self, cfg, o_rows, slot_pos, topk_weights, status=None):
         return torch.from_numpy(oracle.combine_rows(o_rows.numpy(), slot_pos.numpy(), topk_weights.numpy()))
 
     def new_workspace(self, cfg, device):
