@@ -1,15 +1,16 @@
 """Benchmark of the fused FP8 routed-expert MoE layer forward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W]
-                    [--config decode|tiny|prefill|skewed|large|decode_w4a8|prefill_w4a8]
+                    [--config large|tiny|decode|prefill|skewed|decode_w4a8|prefill_w4a8]
                     [--impl reference] [--no-cpu-baseline] [--tokens T] [--shared-expert]
                     [--recipe 0|1|2] [--gate | --gate-only] [--no-graph]
 
 One step = one moe_forward call (route, permute, quantize, gate+up GEMM with SwiGLU and
 requantization, down GEMM, combine) over one batch of seeded synthetic inputs of the named
-problem, inputs resident in HBM.  The default problem is the decode configuration (64 tokens,
-H 2816, I 768, 128 experts, top-8); its ~0.85 GB of FP8 weights exceed the 126 MB L2, so every
-step streams them from HBM.  The timed loop replays a CUDA graph of 10 steps (--no-graph:
+problem, inputs resident in HBM.  The default problem is the largest one that fits one GPU, the
+large prefill with biases (16384 tokens, H 4096, I 1536, 128 experts, top-8, 4.95 TFLOP per step);
+its 2.4 GB of FP8 weights exceed the 126 MB L2, so every step streams them from HBM (likewise
+decode, prefill and the W4A8 problems).  The timed loop replays a CUDA graph of 10 steps (--no-graph:
 host launches); the e2e figure copies each step's inputs in and its output out through pinned
 host memory, on copy streams that overlap the neighbouring steps.  --gate starts every step from
 the gate (moe_gate) instead of router logits; --gate-only times the gate alone.
@@ -76,6 +77,49 @@ def describe(shape: synth.Shape) -> str:
             f"E {shape.num_experts}, top-{shape.top_k}, {rt}" + (", " + ", ".join(extra) if extra else "")
             + (" + 1 shared expert" if shape.shared_experts else "")
             + f"; {rec}")
+
+
+def workload_config(shape, active, world, gate=False):
+    """The `config` object of the JSON line, the same for the native and the reference arm."""
+    alg = algorithmic_bytes(shape, active)
+    return {"workload": describe(shape) + ("; from bf16 hidden states through the fused gate "
+                                           "(RMSNorm + router matmul + top-k)" if gate else ""),
+            "tokens_per_step": shape.num_tokens, "active_experts": active,
+            "parallelism": f"replicas x{world}",
+            "l2": "no flush; the step streams the FP8 weights, larger than L2" if alg > 126e6
+                  else "working set fits L2 (latency-bound)"}
+
+
+def host_sample(prob, n, seed=7):
+    """A host copy of the problem cut to n seeded tokens (every weight, the sampled rows of x and
+    the logits): the oracle's input for the CPU baseline.  Valid as a sample of the whole batch
+    because a row's output does not depend on the other rows."""
+    T = prob.shape.num_tokens
+    tok = np.sort(np.random.default_rng(seed).choice(T, n, replace=False))
+    ti = torch.from_numpy(tok).to(prob.x.device)
+    cpu = lambda t: None if t is None else t.cpu()
+    return synth.Problem(prob.shape.with_tokens(n), prob.x[ti].cpu(), prob.logits[ti].cpu(),
+                         cpu(prob.per_expert_scale), cpu(prob.w13), cpu(prob.w13_scale), cpu(prob.w2),
+                         cpu(prob.w2_scale), cpu(prob.w13_bias), cpu(prob.w2_bias))
+
+
+def time_cpu_oracle(shape, prob, n, budget_s, threads=None, max_reps=50):
+    """Repeat the oracle on n tokens until budget_s seconds have passed: (tokens/s, seconds,
+    runs, threads used)."""
+    import oracle
+    before = oracle.num_threads()
+    done = tot = 0.0
+    reps = 0
+    try:
+        while tot < budget_s and reps < max_reps:
+            _, dt, cores = run_cpu_oracle(shape, prob, n, threads)
+            tot += dt
+            done += n
+            reps += 1
+    finally:
+        if threads:
+            oracle.set_num_threads(before)
+    return done / tot, tot, reps, cores
 
 
 def flops(shape, A):
@@ -332,7 +376,11 @@ def ep_bench(args, shape, world, rank, local, dist):
 def reference_arm(args, shape, rank):
     if rank != 0:
         return
+    import oracle
     prob = synth.make_problem(shape, device="cpu")
+    idx, _, _ = oracle.route(oracle.Config(**shape.cfg()), prob.numpy_inputs()["logits"],
+                             prob.numpy_inputs()["per_expert_scale"])
+    active = int(np.unique(idx).size) + shape.shared_experts
     # tokens per step: the whole batch where one oracle call on it takes well under a second
     # (tiny, decode), else a sample sized so that a step stays near a second
     n = {"tiny": 16, "decode": 64, "decode_w4a8": 64, "skewed": 16, "prefill": 2, "large": 4}.get(shape.name, 4)
@@ -344,11 +392,12 @@ def reference_arm(args, shape, rank):
         times.append(dt)
     tot = sum(times)
     value = n * args.steps / tot
-    sample = f"{n} of {shape.num_tokens} tokens per step (a row's output does not depend on other rows)"
+    sample = (f"{n} of {shape.num_tokens} tokens per step, evenly spaced (a row's output does not depend on "
+              f"the other rows)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": describe(shape), "tokens_per_step": n},
+            "data": "synthetic", "config": workload_config(shape, active, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -360,7 +409,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="decode", choices=sorted(synth.SHAPES))
+    ap.add_argument("--config", default="large", choices=sorted(synth.SHAPES))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
@@ -434,8 +483,15 @@ def main():
     d = prob.to(dev)
     cfg = moe.Config(**shape.cfg())
     weights = moe.transform_weights(cfg, d.w13, d.w13_scale, d.w2, d.w2_scale)
+    # the CPU baseline's input: a host copy of a token sample with every weight, taken before the
+    # device copies of the big problems' untransformed weights are freed
+    cpu_n = {"tiny": 16, "decode": 64, "skewed": 64, "prefill": 4, "large": 16}.get(shape.name, 8)
+    cpu_prob = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu_prob = prob if prob.x.device.type == "cpu" and cpu_n >= shape.num_tokens else \
+            host_sample(prob, min(cpu_n, shape.num_tokens))
     if big:
-        del d.w13, d.w2
+        del d.w13, d.w2, prob
     ws = moe.new_workspace(cfg, dev)
     y = torch.empty((shape.num_tokens, shape.hidden), dtype=torch.bfloat16, device=dev)
     counts = torch.zeros(shape.num_experts + shape.shared_experts, dtype=torch.int32, device=dev)
@@ -636,7 +692,9 @@ def main():
     if rank == 0:
         pk, pk_kind = peaks()
         hbm = float(pk["hbm_gbs"])
-        fp8_peak = float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])) * FP8_OVER_BF16
+        # dense FP8 peak: the measured burst bf16 GEMM rate x the nominal FP8/BF16 ratio (the
+        # higher, stricter denominator of the two measured bf16 figures)
+        fp8_peak = float(pk["bf16_tflops"]) * FP8_OVER_BF16
         tok_s = job_tokens_per_s(world, shape.num_tokens, args.steps, ms)
         per_step_s = ms / 1e3 / args.steps
         fl = flops(shape, A)
@@ -661,19 +719,14 @@ def main():
                 ("k_grouped_gemm_narrow" if few else "k_grouped_gemm")
         roof.update({"kernel": kname + "<gate+up>",
                      "traffic": traffic_for("gemm1", shape.name),
-                     "peak_source": f"{pk_kind} ({'sustained bf16 x2 for fp8' if compute_bound else 'copy'})",
+                     "peak_source": f"{pk_kind} ({'burst bf16 x2 for fp8' if compute_bound else 'copy'})",
                      "algorithmic_bytes_per_launch": g1_bytes, "ms_per_launch": g1_ms})
         layer_roof_s = max(fl / (fp8_peak * 1e12), alg / (hbm * 1e9))
         line = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
-            "config": {"workload": describe(shape) + ("; from bf16 hidden states through the fused gate "
-                                                      "(RMSNorm + router matmul + top-k)" if args.gate else ""),
-                       "tokens_per_step": shape.num_tokens,
-                       "active_experts": active, "parallelism": f"replicas x{world}",
-                       "l2": "no flush; the step streams the FP8 weights, larger than L2" if alg > 126e6
-                             else "working set fits L2 (latency-bound)"},
+            "config": workload_config(shape, active, world, args.gate),
             "tflops": fl / per_step_s / 1e12,
             "layer_roofline": {"bound": "tensor" if compute_bound else "hbm", "roofline_ms": layer_roof_s * 1e3,
                                "frac": layer_roof_s / per_step_s, "algorithmic_bytes": alg, "flops": fl},
@@ -698,21 +751,19 @@ def main():
                             "GB/s": gbytes / (gate_ms / 1e3) / 1e9, "TFLOP/s": gflops / (gate_ms / 1e3) / 1e12,
                             "note": "stages_ms covers the forward after the gate (its route stage is "
                                     "empty: the routing comes from the gate)"}
-        if world == 1 and not args.no_cpu_baseline:
-            n = {"tiny": 16, "decode": 64, "skewed": 64, "prefill": 4, "large": 16}.get(shape.name, 8)
-            cpu_prob = prob if prob.x.device.type == "cpu" else None
-            if cpu_prob is not None:
-                done = tot = 0.0
-                reps = 0
-                while tot < 5.0 and reps < 50:
-                    v, dt, cores = run_cpu_oracle(shape, cpu_prob, n)
-                    tot += dt
-                    done += n
-                    reps += 1
-                line["cpu_baseline"] = {"value": done / tot, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                        "sample": f"{n} of {shape.num_tokens} tokens x {reps} runs, {tot:.1f} s"}
-            else:
-                line["cpu_baseline"] = None
+        if cpu_prob is not None:
+            n = cpu_prob.shape.num_tokens
+            v, tot, reps, cores = time_cpu_oracle(cpu_prob.shape, cpu_prob, n, 10.0)
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                    "sample": f"{n} of {shape.num_tokens} tokens (seeded sample, every "
+                                              f"weight) x {reps} runs, {tot:.1f} s"}
+            if shape.name in ("tiny", "decode"):
+                v1, tot1, reps1, _ = time_cpu_oracle(cpu_prob.shape, cpu_prob, n, 5.0, threads=1)
+                line["cpu_baseline_1thread"] = {"value": v1, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                                "sample": f"{n} of {shape.num_tokens} tokens x {reps1} runs, "
+                                                          f"{tot1:.1f} s"}
+        elif world == 1:
+            line["cpu_baseline"] = None
         print(json.dumps(line), flush=True)
 
     if dist:
