@@ -36,6 +36,18 @@ class LibraryOps:
         if moe_module is None:
             import mixture_experts_fp8_b200 as moe_module
         self.moe = moe_module
+        self._rows_ws = {}          # device -> the expert side's workspace (grows, never shrinks)
+
+    def rows_workspace(self, cfg_rows, device):
+        """A workspace for the expert-side problem cfg_rows, kept from step to step: the row
+        count varies per step, so the buffer grows to the largest problem seen and is reused (the
+        steps run in stream order, so one buffer serves them all)."""
+        need = self.moe.workspace_size(cfg_rows)
+        ws = self._rows_ws.get(str(device))
+        if ws is None or ws.numel() < need:
+            ws = self.moe.new_workspace(cfg_rows, device)
+            self._rows_ws[str(device)] = ws
+        return ws
 
     def route(self, cfg, router_logits, per_expert_scale):
         return self.moe.route(cfg, router_logits, per_expert_scale=per_expert_scale)
@@ -45,7 +57,7 @@ class LibraryOps:
 
     def rows(self, cfg_rows, rows, expert_of_row, weights_local, w13_bias, w2_bias):
         return self.moe.forward_rows(cfg_rows, rows, expert_of_row, weights_local, w13_bias=w13_bias,
-                                     w2_bias=w2_bias)
+                                     w2_bias=w2_bias, workspace=self.rows_workspace(cfg_rows, rows.device))
 
     def combine(self, cfg, o_rows, slot_pos, topk_weights, status=None):
         return self.moe.combine_rows(cfg, o_rows, slot_pos, topk_weights, status=status)
@@ -57,6 +69,17 @@ class LibraryOps:
         """The dispatch's status word (device int32 [1]: the first word of the workspace)."""
         import torch
         return workspace[:4].view(torch.int32)
+
+
+_LIBRARY_OPS = None
+
+
+def _library_ops():
+    """One LibraryOps per process, so that its expert-side workspace outlives a step."""
+    global _LIBRARY_OPS
+    if _LIBRARY_OPS is None:
+        _LIBRARY_OPS = LibraryOps()
+    return _LIBRARY_OPS
 
 
 def rows_config(cfg, ranks: int, n_rows: int):
@@ -84,7 +107,7 @@ def ep_step(cfg, ranks: int, x, router_logits, weights_local, dist, group=None, 
     [T, E] in, y [T, H] (bf16) out.  cfg: this rank's tokens and the global expert count;
     weights_local: moe.transform_weights of this rank's E/R experts.  Returns (y, stats)."""
     import torch
-    ops = ops or LibraryOps()
+    ops = ops or _library_ops()
     dev = x.device
     if workspace is None:
         workspace = ops.new_workspace(cfg, dev)

@@ -185,3 +185,29 @@ def test_one_rank_with_the_benchmark_local_exchange():
                          logits=ni["logits"], per_expert_scale=ni["per_expert_scale"], b13=ni["b13"], b2=ni["b2"])
     assert np.array_equal(y.numpy(), ref)
     assert stats["sent"] == stats["received"] == [shape.num_tokens * shape.top_k]
+
+
+def test_library_ops_keep_one_growing_expert_side_workspace():
+    """The expert side's workspace is kept across steps: reused while the step's problem fits,
+    replaced by a larger one when it does not, never shrunk (host logic, a fake library)."""
+    from mixture_experts_fp8_b200 import ep
+
+    class FakeMoe:
+        def __init__(self):
+            self.made = []
+
+        def workspace_size(self, cfg):
+            return 1000 * cfg.num_tokens
+
+        def new_workspace(self, cfg, device):
+            ws = torch.empty(self.workspace_size(cfg), dtype=torch.uint8, device=device)
+            self.made.append(ws.numel())
+            return ws
+
+    import mixture_experts_fp8_b200 as moe
+    cfg = moe.Config(**synth.SHAPES["tiny"].cfg())
+    fake = FakeMoe()
+    ops = ep.LibraryOps(fake)
+    sizes = [ops.rows_workspace(ep.rows_config(cfg, 1, n), "cpu").numel() for n in [40, 12, 40, 64, 8, 64]]
+    assert fake.made == [40000, 64000]
+    assert sizes == [40000, 40000, 40000, 64000, 64000, 64000]
