@@ -183,3 +183,38 @@ def test_forward_rows_rejects_more_than_one_slot():
     w = tuple(torch.zeros(n, dtype=torch.uint8, device="cuda") for n in moe.transformed_weights_size(cfg))
     with pytest.raises(moe.MoeError):
         moe.forward_rows(cfg, x, e, w)
+
+
+class _OneRank:
+    """The all-to-all of a single rank: every row stays home."""
+
+    @staticmethod
+    def all_to_all_single(out, inp, out_splits=None, in_splits=None, group=None):
+        out.copy_(inp)
+
+
+@pytest.mark.parametrize("name", ["tiny_r0", "w4a8"])
+def test_ep_step_through_the_library_ops_equals_the_forward(name):
+    """ep_step with its default device steps (the library ops, which keep one expert-side
+    workspace from call to call) at one rank: the same bits as the fused forward, for the whole
+    batch and then for a smaller one through the kept workspace."""
+    moe = _lib()
+    from mixture_experts_fp8_b200 import ep
+    shape = SHAPES[name]
+    d = synth.make_problem(shape).to("cuda")
+    full = moe.Config(**shape.cfg())
+    w = moe.transform_weights(full, d.w13, d.w13_scale, d.w2, d.w2_scale)
+    for T in (shape.num_tokens, shape.num_tokens // 2, shape.num_tokens):
+        cfg = replace(full, num_tokens=T)
+        x, logits = d.x[:T].contiguous(), d.logits[:T].contiguous()
+        y_ep, stats = ep.ep_step(cfg, 1, x, logits, w, _OneRank(), per_expert_scale=d.per_expert_scale,
+                                 w13_bias_local=d.w13_bias, w2_bias_local=d.w2_bias)
+        y_f = moe.forward(cfg, x, w, router_logits=logits, per_expert_scale=d.per_expert_scale,
+                          w13_bias=d.w13_bias, w2_bias=d.w2_bias)
+        torch.cuda.synchronize()
+        assert stats["sent"] == [T * shape.top_k] and stats["received"] == [T * shape.top_k]
+        assert torch.equal(y_ep.view(torch.int16), y_f.view(torch.int16)), f"{name}, {T} tokens"
+    kept = ep._library_ops()._rows_ws
+    assert len(kept) == 1
+    need = moe.workspace_size(ep.rows_config(full, 1, shape.num_tokens * shape.top_k))
+    assert next(iter(kept.values())).numel() >= need
