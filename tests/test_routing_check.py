@@ -92,3 +92,42 @@ def test_choice_spanning_too_many_groups_is_rejected():
     assert not ok and "groups" in why
     ok, _ = near_tie_choice_ok(c, LOGITS[0], g, [0, 4, 9][:2] + [5])
     assert ok                               # groups {0, 1}: 0, 4, 5
+
+
+def _closed_form_weights(logits, ids, routing, renormalize, pes, rsf):
+    """The weight rule written out in fp64 ("MindIE-SD Fused MoE", routing parameters): softmax
+    over every expert, or over the chosen ones when renormalized; sigmoid scores always divided by
+    their sum; then the per-expert scale, then the routed scaling factor."""
+    l = logits.astype(np.float64)
+    if routing == 0:
+        e = np.exp(l - l.max())
+        w = e[ids] / (e[ids].sum() if renormalize else e.sum())
+    else:
+        s = 1.0 / (1.0 + np.exp(-l))
+        w = s[ids] / s[ids].sum()
+    if pes is not None:
+        w = w * pes.astype(np.float64)[ids]
+    return w * rsf
+
+
+@pytest.mark.parametrize("routing,renormalize,use_pes,rsf", [
+    (1, 1, False, 1.0), (1, 1, True, 2.5), (0, 1, False, 1.0), (0, 0, True, 1.0), (0, 1, True, 2.5)])
+def test_route_weights_match_the_closed_form_for_a_choice_the_oracle_would_not_make(routing, renormalize,
+                                                                                    use_pes, rsf):
+    shape = synth.Shape("w", 1, 128, 128, 16, 3, routing=routing, renormalize=renormalize,
+                        routed_scaling_factor=rsf)
+    c = oracle.Config(**shape.cfg())
+    pes = np.linspace(0.5, 1.5, 16).astype(np.float32) if use_pes else None
+    ids = np.array([[9, 2, 13]], np.int32)          # not the top 3 of LOGITS
+    w = oracle.route_weights(c, LOGITS, ids, pes)
+    np.testing.assert_allclose(w[0], _closed_form_weights(LOGITS[0], ids[0], routing, renormalize, pes, rsf),
+                               rtol=2e-6)
+
+
+def test_group_scores_top2_sum():
+    """group_select_mode 1: a group scores the sum of its two best sigmoid scores."""
+    shape = synth.Shape("g1", 1, 128, 128, 16, 2, routing=1, renormalize=1, group_count=4, k_group=2,
+                        group_select_mode=1)
+    g = oracle.group_scores(oracle.Config(**shape.cfg()), LOGITS)[0]
+    s = np.sort(1.0 / (1.0 + np.exp(-LOGITS[0].astype(np.float64))).reshape(4, 4), axis=1)
+    np.testing.assert_allclose(g, s[:, -1] + s[:, -2], rtol=1e-6)
